@@ -1,0 +1,280 @@
+"""Python binding of the sm_100a paged latent-attention library (``libmla_b200.so``).
+
+Argument marshalling only: torch tensors give device pointers and the current CUDA
+stream; host index tables are copied into int32 arrays.  Every step of the attention
+runs in the library's CUDA kernels.  If the library is missing the calls raise; there
+is no other implementation to fall back to.
+
+Names follow the C ABI in ``include/mla.h``: ``mla_supports``, ``mla_plan``,
+``mla_run``, ``mla_plan_check``, ``mla_plan_get_info``, ``mla_plan_describe``,
+``mla_plan_destroy``, ``mla_status_string``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmla_b200.so")
+
+MLA_OK = 0
+MLA_ERR_INVALID_ARGUMENT = 1
+MLA_ERR_UNSUPPORTED = 2
+MLA_ERR_CUDA = 3
+MLA_ERR_OUT_OF_MEMORY = 4
+MLA_ERR_DEVICE_TIMEOUT = 5
+MLA_DEBUG_DROP_FIRST_KV_LOAD = 1
+WORK_FIELDS = 8
+MERGE_FIELDS = 4
+KV_LORA_RANK = 512
+ROPE_DIM = 64
+
+EXPORTED = (
+    "mla_supports",
+    "mla_plan",
+    "mla_run",
+    "mla_plan_check",
+    "mla_plan_get_info",
+    "mla_plan_describe",
+    "mla_plan_destroy",
+    "mla_status_string",
+)
+
+
+class MlaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [
+        ("num_heads", ctypes.c_int32),
+        ("kv_lora_rank", ctypes.c_int32),
+        ("rope_dim", ctypes.c_int32),
+        ("page_size", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32),
+        ("sm_scale", ctypes.c_float),
+    ]
+
+
+class _Options(ctypes.Structure):
+    _fields_ = [
+        ("split_keys", ctypes.c_int32),
+        ("num_sms", ctypes.c_int32),
+        ("wait_timeout_ns", ctypes.c_uint64),
+        ("debug_flags", ctypes.c_int32),
+        ("host_only", ctypes.c_int32),
+    ]
+
+
+class _Info(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("total_tokens", ctypes.c_int32),
+        ("num_work", ctypes.c_int32),
+        ("num_merge", ctypes.c_int32),
+        ("num_partials", ctypes.c_int32),
+        ("num_sms", ctypes.c_int32),
+        ("workspace_bytes", ctypes.c_int64),
+    ]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load (once) and return the library; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"CUDA library {path} is missing: build it with "
+            "`python -m paged_head_latent_mla_b200._build` (there is no fallback)")
+    lib = ctypes.CDLL(path)
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    vp = ctypes.c_void_p
+    lib.mla_supports.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    lib.mla_supports.restype = ctypes.c_int
+    lib.mla_plan.argtypes = [ctypes.POINTER(_Dims), ctypes.c_int32, i32p, i32p, i32p, i32p, ctypes.c_int32, vp,
+                             ctypes.POINTER(_Options), ctypes.POINTER(vp)]
+    lib.mla_plan.restype = ctypes.c_int
+    lib.mla_run.argtypes = [vp, vp, vp, vp, vp, vp, vp]
+    lib.mla_run.restype = ctypes.c_int
+    lib.mla_plan_check.argtypes = [vp]
+    lib.mla_plan_check.restype = ctypes.c_int
+    lib.mla_plan_get_info.argtypes = [vp, ctypes.POINTER(_Info)]
+    lib.mla_plan_get_info.restype = ctypes.c_int
+    lib.mla_plan_describe.argtypes = [vp, i32p, i32p, i32p]
+    lib.mla_plan_describe.restype = ctypes.c_int
+    lib.mla_plan_destroy.argtypes = [vp]
+    lib.mla_plan_destroy.restype = None
+    lib.mla_status_string.argtypes = [ctypes.c_int]
+    lib.mla_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().mla_status_string(int(status)).decode()
+
+
+mla_status_string = status_string
+
+
+def _i32(x) -> np.ndarray:
+    try:
+        import torch
+
+        if isinstance(x, torch.Tensor):
+            if x.is_cuda:
+                raise ValueError("page tables are host arrays (CPU tensors, numpy arrays or lists)")
+            x = x.numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.int32))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+def mla_supports(kv_lora_rank: int, rope_dim: int, num_heads: int, page_size: int) -> bool:
+    return bool(load_library().mla_supports(kv_lora_rank, rope_dim, num_heads, page_size))
+
+
+class MlaPlan:
+    """Owns one C plan handle (``mla_plan_t``); destroyed with the object."""
+
+    def __init__(self, handle: int, batch: int, num_heads: int, total_tokens: int):
+        self._h = ctypes.c_void_p(handle)
+        self.batch = batch
+        self.num_heads = num_heads
+        self.total_tokens = total_tokens
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        if not self._h:
+            raise RuntimeError("plan was destroyed")
+        return self._h
+
+    def destroy(self) -> None:
+        if self._h:
+            load_library().mla_plan_destroy(self._h)
+            self._h = ctypes.c_void_p(None)
+
+    def __del__(self):  # pragma: no cover - interpreter shutdown order
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+def mla_plan(qo_indptr, kv_indptr, kv_indices, last_page_len, *, num_heads: int, page_size: int, num_pages: int,
+             sm_scale: float, causal: bool = True, kv_lora_rank: int = KV_LORA_RANK, rope_dim: int = ROPE_DIM,
+             split_keys: int = 0, num_sms: int = 0, wait_timeout_ns: int = 0, debug_flags: int = 0,
+             host_only: bool = False, stream=None) -> MlaPlan:
+    """Plan one step from host page tables (``mla_plan``)."""
+    lib = load_library()
+    qo = _i32(qo_indptr)
+    kvp = _i32(kv_indptr)
+    kvi = _i32(kv_indices)
+    last = _i32(last_page_len)
+    batch = len(qo) - 1
+    if batch < 0 or len(kvp) != batch + 1 or len(last) != batch:
+        raise MlaError(MLA_ERR_INVALID_ARGUMENT, "mla_plan: table lengths")
+    if len(kvi) < int(kvp[-1]):
+        raise MlaError(MLA_ERR_INVALID_ARGUMENT, "mla_plan: kv_indices shorter than kv_indptr[-1]")
+    dims = _Dims(num_heads, kv_lora_rank, rope_dim, page_size, num_pages, sm_scale)
+    opts = _Options(split_keys, num_sms, wait_timeout_ns, debug_flags, 1 if host_only else 0)
+    if stream is None and not host_only:
+        import torch
+
+        stream = torch.cuda.current_stream().cuda_stream
+    out = ctypes.c_void_p()
+    kvi_arr = kvi if len(kvi) else np.zeros(1, dtype=np.int32)
+    st = lib.mla_plan(ctypes.byref(dims), batch, _ptr(qo), _ptr(kvp), _ptr(kvi_arr), _ptr(last),
+                      1 if causal else 0, ctypes.c_void_p(stream or 0), ctypes.byref(opts), ctypes.byref(out))
+    if st != MLA_OK:
+        raise MlaError(st, "mla_plan")
+    return MlaPlan(out.value, batch, num_heads, int(qo[-1]))
+
+
+def mla_plan_get_info(plan: MlaPlan) -> dict:
+    info = _Info()
+    st = load_library().mla_plan_get_info(plan.handle, ctypes.byref(info))
+    if st != MLA_OK:
+        raise MlaError(st, "mla_plan_get_info")
+    return {f: getattr(info, f) for f, _ in _Info._fields_}
+
+
+def mla_plan_describe(plan: MlaPlan) -> dict:
+    """kv_len [B], work [num_work, 8] and merge [num_merge, 4] as int32 arrays."""
+    info = mla_plan_get_info(plan)
+    kv_len = np.zeros(max(1, info["batch"]), dtype=np.int32)
+    work = np.zeros((max(1, info["num_work"]), WORK_FIELDS), dtype=np.int32)
+    merge = np.zeros((max(1, info["num_merge"]), MERGE_FIELDS), dtype=np.int32)
+    st = load_library().mla_plan_describe(plan.handle, _ptr(kv_len), _ptr(work), _ptr(merge))
+    if st != MLA_OK:
+        raise MlaError(st, "mla_plan_describe")
+    return {
+        "kv_len": kv_len[: info["batch"]],
+        "work": work[: info["num_work"]],
+        "merge": merge[: info["num_merge"]],
+        "info": info,
+    }
+
+
+def _check_dev_tensor(t, name, dtype, shape):
+    import torch
+
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def mla_run(plan: MlaPlan, q_nope, q_pe, cache, out=None, lse=None, return_lse: bool = False, stream=None):
+    """Run the planned attention (``mla_run``).  Returns ``out`` or ``(out, lse)``."""
+    import torch
+
+    T, H = plan.total_tokens, plan.num_heads
+    _check_dev_tensor(q_nope, "q_nope", torch.bfloat16, (T, H, KV_LORA_RANK))
+    _check_dev_tensor(q_pe, "q_pe", torch.bfloat16, (T, H, ROPE_DIM))
+    if cache.dim() != 3 or cache.shape[-1] != KV_LORA_RANK + ROPE_DIM:
+        raise ValueError("cache must be [num_pages, page_size, 576]")
+    _check_dev_tensor(cache, "cache", torch.bfloat16, tuple(cache.shape))
+    if out is None:
+        out = torch.empty((T, H, KV_LORA_RANK), dtype=torch.bfloat16, device=q_nope.device)
+    _check_dev_tensor(out, "out", torch.bfloat16, (T, H, KV_LORA_RANK))
+    if return_lse and lse is None:
+        lse = torch.empty((T, H), dtype=torch.float32, device=q_nope.device)
+    if lse is not None:
+        _check_dev_tensor(lse, "lse", torch.float32, (T, H))
+    if stream is None:
+        stream = torch.cuda.current_stream(q_nope.device).cuda_stream
+    st = load_library().mla_run(plan.handle, ctypes.c_void_p(q_nope.data_ptr()), ctypes.c_void_p(q_pe.data_ptr()),
+                                ctypes.c_void_p(cache.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+                                ctypes.c_void_p(lse.data_ptr() if lse is not None else 0),
+                                ctypes.c_void_p(stream or 0))
+    if st != MLA_OK:
+        raise MlaError(st, "mla_run")
+    return (out, lse) if (return_lse or lse is not None) else out
+
+
+def mla_plan_check(plan: MlaPlan) -> int:
+    """Wait for the plan's last run; return its device status (0 = ok)."""
+    return int(load_library().mla_plan_check(plan.handle))
+
+
+def mla_plan_destroy(plan: MlaPlan) -> None:
+    plan.destroy()

@@ -1,0 +1,265 @@
+// C ABI of the paged latent-attention library: plan ownership, tensor-map encoding,
+// launches and the device status word.  See include/mla.h for the contract.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "mla_internal.h"
+
+#include "mla_launch.h"
+
+using namespace mla;
+
+struct mla_plan_s {
+  mla_dims dims{};
+  int32_t batch = 0;
+  bool causal = true;
+  mla_plan_options opts{};
+  PlanLayout layout;
+  int device = -1;
+  bool host_only = false;
+  // one device blob: [status (256 B)] [work] [merge] [kv_indices]
+  void* d_blob = nullptr;
+  int32_t* d_status = nullptr;
+  WorkItem* d_work = nullptr;
+  MergeItem* d_merge = nullptr;
+  int32_t* d_kv_indices = nullptr;
+  float* d_ws = nullptr;  // [partials * 128 * 512] o, then [partials * 128] lse
+  void* h_staging = nullptr;
+  cudaEvent_t ev_last = nullptr;
+};
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix with row pitch `pitch_elems`.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_elems,
+              uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {pitch_elems * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+void free_plan(mla_plan_s* p) {
+  if (!p) return;
+  if (!p->host_only) {
+    if (p->ev_last) {
+      cudaEventSynchronize(p->ev_last);
+      cudaEventDestroy(p->ev_last);
+    }
+    if (p->d_blob) cudaFree(p->d_blob);
+    if (p->d_ws) cudaFree(p->d_ws);
+    if (p->h_staging) cudaFreeHost(p->h_staging);
+  }
+  delete p;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mla_supports(int kv_lora_rank, int rope_dim, int num_heads, int page_size) {
+  return shape_supported(kv_lora_rank, rope_dim, num_heads, page_size) ? 1 : 0;
+}
+
+const char* mla_status_string(mla_status s) {
+  switch (s) {
+    case MLA_OK: return "ok";
+    case MLA_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case MLA_ERR_UNSUPPORTED: return "unsupported shape";
+    case MLA_ERR_CUDA: return "CUDA error";
+    case MLA_ERR_OUT_OF_MEMORY: return "out of memory";
+    case MLA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+mla_status mla_plan(const mla_dims* dims, int32_t batch, const int32_t* qo_indptr, const int32_t* kv_indptr,
+                    const int32_t* kv_indices, const int32_t* last_page_len, int32_t causal, void* stream,
+                    const mla_plan_options* opts, mla_plan_t* out_plan) {
+  if (!out_plan) return MLA_ERR_INVALID_ARGUMENT;
+  *out_plan = nullptr;
+  if (!dims || (causal != 0 && causal != 1)) return MLA_ERR_INVALID_ARGUMENT;
+  mla_plan_s* p = new (std::nothrow) mla_plan_s();
+  if (!p) return MLA_ERR_OUT_OF_MEMORY;
+  p->dims = *dims;
+  p->batch = batch;
+  p->causal = causal != 0;
+  if (opts) p->opts = *opts;
+  p->host_only = p->opts.host_only != 0;
+
+  int num_sms = p->opts.num_sms;
+  if (!p->host_only) {
+    if (cudaGetDevice(&p->device) != cudaSuccess) { free_plan(p); return MLA_ERR_CUDA; }
+    if (num_sms <= 0) {
+      if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, p->device) != cudaSuccess) {
+        free_plan(p);
+        return MLA_ERR_CUDA;
+      }
+    }
+  } else if (num_sms <= 0) {
+    num_sms = 148;
+  }
+  p->opts.num_sms = num_sms;
+
+  mla_status st = build_layout(*dims, batch, qo_indptr, kv_indptr, kv_indices, last_page_len, p->causal,
+                               p->opts.split_keys, num_sms, &p->layout);
+  if (st != MLA_OK) { free_plan(p); return st; }
+  if (p->host_only) { *out_plan = p; return MLA_OK; }
+
+  // ---- device buffers owned by the plan, uploaded through plan-owned pinned staging
+  const size_t n_idx = batch > 0 ? static_cast<size_t>(kv_indptr[batch]) : 0;
+  const size_t off_work = 256;
+  const size_t off_merge = align_up(off_work + sizeof(WorkItem) * p->layout.work.size(), 256);
+  const size_t off_idx = align_up(off_merge + sizeof(MergeItem) * p->layout.merge.size(), 256);
+  const size_t blob = align_up(off_idx + sizeof(int32_t) * n_idx, 256);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMalloc(&p->d_blob, blob) != cudaSuccess) { cudaGetLastError(); free_plan(p); return MLA_ERR_OUT_OF_MEMORY; }
+  if (cudaMallocHost(&p->h_staging, blob) != cudaSuccess) { cudaGetLastError(); free_plan(p); return MLA_ERR_OUT_OF_MEMORY; }
+  uint8_t* h = static_cast<uint8_t*>(p->h_staging);
+  std::memset(h, 0, off_work);
+  if (!p->layout.work.empty()) std::memcpy(h + off_work, p->layout.work.data(), sizeof(WorkItem) * p->layout.work.size());
+  if (!p->layout.merge.empty())
+    std::memcpy(h + off_merge, p->layout.merge.data(), sizeof(MergeItem) * p->layout.merge.size());
+  if (n_idx) std::memcpy(h + off_idx, kv_indices, sizeof(int32_t) * n_idx);
+  uint8_t* d = static_cast<uint8_t*>(p->d_blob);
+  p->d_status = reinterpret_cast<int32_t*>(d);
+  p->d_work = reinterpret_cast<WorkItem*>(d + off_work);
+  p->d_merge = reinterpret_cast<MergeItem*>(d + off_merge);
+  p->d_kv_indices = reinterpret_cast<int32_t*>(d + off_idx);
+  if (p->layout.num_partials > 0) {
+    const size_t ws = static_cast<size_t>(p->layout.num_partials) * kTileM * (kCkv + 1) * sizeof(float);
+    if (cudaMalloc(&p->d_ws, ws) != cudaSuccess) { cudaGetLastError(); free_plan(p); return MLA_ERR_OUT_OF_MEMORY; }
+  }
+  if (cudaEventCreateWithFlags(&p->ev_last, cudaEventDisableTiming) != cudaSuccess ||
+      cudaMemcpyAsync(p->d_blob, p->h_staging, blob, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaEventRecord(p->ev_last, s) != cudaSuccess) {
+    cudaGetLastError();
+    free_plan(p);
+    return MLA_ERR_CUDA;
+  }
+  *out_plan = p;
+  return MLA_OK;
+}
+
+mla_status mla_run(mla_plan_t p, const void* q_nope, const void* q_pe, const void* cache, void* out, float* lse,
+                   void* stream) {
+  if (!p || p->host_only) return MLA_ERR_INVALID_ARGUMENT;
+  const int64_t rows = static_cast<int64_t>(p->layout.total_tokens) * p->dims.num_heads;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (p->layout.work.empty()) return MLA_OK;
+  if (!q_nope || !q_pe || !cache || !out) return MLA_ERR_INVALID_ARGUMENT;
+  auto misaligned = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) != 0; };
+  if (misaligned(q_nope) || misaligned(q_pe) || misaligned(cache) || misaligned(out) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return MLA_ERR_INVALID_ARGUMENT;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != p->device) return MLA_ERR_INVALID_ARGUMENT;
+
+  const int P = p->dims.page_size;
+  CUtensorMap tm_q, tm_qpe, tm_kv, tm_kpe;
+  const uint64_t cache_rows = static_cast<uint64_t>(p->dims.num_pages) * P;
+  const uint32_t box_rows = P < kTileN ? P : kTileN;
+  if (!make_map(&tm_q, q_nope, rows, kCkv, kCkv, 64, kTileM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tm_qpe, q_pe, rows, kRope, kRope, 32, kTileM, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map(&tm_kv, cache, cache_rows, kLatent, kLatent, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tm_kpe, cache, cache_rows, kLatent, kLatent, 32, box_rows, CU_TENSOR_MAP_SWIZZLE_64B))
+    return MLA_ERR_CUDA;
+
+  AttnParams ap;
+  ap.work = p->d_work;
+  ap.kv_indices = p->d_kv_indices;
+  ap.out = out;
+  ap.lse = lse;
+  ap.ws_o = p->d_ws;
+  ap.ws_lse = p->d_ws ? p->d_ws + static_cast<size_t>(p->layout.num_partials) * kTileM * kCkv : nullptr;
+  ap.status = p->d_status;
+  ap.scale_log2 = p->dims.sm_scale * 1.4426950408889634f;
+  ap.num_heads = p->dims.num_heads;
+  ap.page_size = P;
+  ap.box_rows = static_cast<int32_t>(box_rows);
+  ap.timeout_ns = p->opts.wait_timeout_ns ? p->opts.wait_timeout_ns : 4000000000ull;
+  ap.debug_flags = p->opts.debug_flags;
+  cudaError_t e = launch_attention(tm_q, tm_qpe, tm_kv, tm_kpe, ap, static_cast<int>(p->layout.work.size()), s);
+  if (e != cudaSuccess) return MLA_ERR_CUDA;
+  if (!p->layout.merge.empty()) {
+    MergeParams mp{p->d_merge, ap.ws_o, ap.ws_lse, ap.out, lse};
+    e = launch_merge(mp, static_cast<int>(p->layout.merge.size()), s);
+    if (e != cudaSuccess) return MLA_ERR_CUDA;
+  }
+  if (cudaEventRecord(p->ev_last, s) != cudaSuccess) return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+mla_status mla_plan_check(mla_plan_t p) {
+  if (!p) return MLA_ERR_INVALID_ARGUMENT;
+  if (p->host_only) return MLA_OK;
+  if (cudaEventSynchronize(p->ev_last) != cudaSuccess) return MLA_ERR_CUDA;
+  int32_t st = 0;
+  if (cudaMemcpy(&st, p->d_status, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return MLA_ERR_CUDA;
+  if (st != 0) {
+    // The bits above the low byte name the wait that gave up (diagnostics only).
+    if (std::getenv("MLA_DEBUG_STATUS")) std::fprintf(stderr, "mla: device status word 0x%x\n", st);
+    if (cudaMemset(p->d_status, 0, sizeof(st)) != cudaSuccess) return MLA_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return MLA_ERR_CUDA;
+    return static_cast<mla_status>(st & 0xff);
+  }
+  return MLA_OK;
+}
+
+mla_status mla_plan_get_info(mla_plan_t p, mla_plan_info* info) {
+  if (!p || !info) return MLA_ERR_INVALID_ARGUMENT;
+  info->batch = p->batch;
+  info->total_tokens = p->layout.total_tokens;
+  info->num_work = static_cast<int32_t>(p->layout.work.size());
+  info->num_merge = static_cast<int32_t>(p->layout.merge.size());
+  info->num_partials = p->layout.num_partials;
+  info->num_sms = p->opts.num_sms;
+  info->workspace_bytes = static_cast<int64_t>(p->layout.num_partials) * kTileM * (kCkv + 1) * 4;
+  return MLA_OK;
+}
+
+mla_status mla_plan_describe(mla_plan_t p, int32_t* kv_len, int32_t* work, int32_t* merge) {
+  if (!p) return MLA_ERR_INVALID_ARGUMENT;
+  if (kv_len && p->batch > 0) std::memcpy(kv_len, p->layout.kv_len.data(), sizeof(int32_t) * p->batch);
+  if (work && !p->layout.work.empty())
+    std::memcpy(work, p->layout.work.data(), sizeof(WorkItem) * p->layout.work.size());
+  if (merge && !p->layout.merge.empty())
+    std::memcpy(merge, p->layout.merge.data(), sizeof(MergeItem) * p->layout.merge.size());
+  return MLA_OK;
+}
+
+void mla_plan_destroy(mla_plan_t p) { free_plan(p); }
+
+}  // extern "C"

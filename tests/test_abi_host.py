@@ -1,0 +1,129 @@
+"""Host-side checks of the C-ABI library (no GPU needed): it loads, exports every
+function include/mla.h declares, validates inputs with the documented status codes,
+and plans on the host."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+import paged_head_latent_mla_b200 as M  # noqa: E402
+
+SCALE = 192 ** -0.5
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_library():
+    from paged_head_latent_mla_b200 import _build
+
+    _build.build()
+    return M.load_library()
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "mla.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(mla_[a-z_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_function():
+    lib = M.load_library()
+    names = declared_functions()
+    assert set(names) == set(M.EXPORTED), names
+    for n in names:
+        assert hasattr(lib, n), n
+        assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
+
+
+def test_supports_matrix():
+    assert M.mla_supports(512, 64, 128, 64)
+    for H in (16, 32, 64, 128):
+        for P in (16, 32, 64, 128):
+            assert M.mla_supports(512, 64, H, P)
+    assert not M.mla_supports(512, 0, 128, 64)  # kpe 0 is not implemented here
+    assert not M.mla_supports(256, 64, 128, 64)
+    assert not M.mla_supports(512, 64, 8, 64)
+    assert not M.mla_supports(512, 64, 128, 1)
+    assert not M.mla_supports(512, 64, 128, 48)
+
+
+def test_status_strings():
+    for code in range(6):
+        assert M.status_string(code)
+    assert M.status_string(99) == "unknown status"
+
+
+def _plan(**kw):
+    args = dict(qo_indptr=[0, 1, 3], kv_indptr=[0, 2, 5], kv_indices=[0, 1, 2, 3, 4], last_page_len=[5, 16],
+                num_heads=16, page_size=16, num_pages=8, sm_scale=SCALE, host_only=True)
+    args.update(kw)
+    return M.mla_plan(**args)
+
+
+def test_host_plan_basic():
+    p = _plan()
+    d = M.mla_plan_describe(p)
+    assert list(d["kv_len"]) == [21, 48]
+    assert d["info"]["total_tokens"] == 3
+    assert d["info"]["num_sms"] == 148
+    p.destroy()
+
+
+@pytest.mark.parametrize(
+    "bad",
+    [
+        dict(qo_indptr=[1, 1, 3]),  # [0] != 0
+        dict(qo_indptr=[0, 2, 1]),  # decreasing
+        dict(kv_indptr=[0, 3, 2]),
+        dict(kv_indices=[0, 1, 2, 3, 8]),  # page id out of range
+        dict(kv_indices=[0, 1, 2, 3, -1]),
+        dict(last_page_len=[0, 16]),  # row with pages needs >= 1
+        dict(last_page_len=[5, 17]),
+        dict(num_pages=0),
+        dict(split_keys=100),  # not a multiple of 64
+        dict(sm_scale=float("nan")),
+    ],
+)
+def test_invalid_arguments(bad):
+    with pytest.raises(M.MlaError) as e:
+        _plan(**bad)
+    assert e.value.status == M.MLA_ERR_INVALID_ARGUMENT
+
+
+@pytest.mark.parametrize("bad", [dict(num_heads=8), dict(page_size=8), dict(kv_lora_rank=256),
+                                 dict(rope_dim=0), dict(num_heads=96)])
+def test_unsupported_shapes(bad):
+    with pytest.raises(M.MlaError) as e:
+        _plan(**bad)
+    assert e.value.status == M.MLA_ERR_UNSUPPORTED
+
+
+def test_empty_row_may_have_zero_last_page_len():
+    p = _plan(kv_indptr=[0, 0, 3], kv_indices=[0, 1, 2], last_page_len=[0, 4])
+    assert list(M.mla_plan_describe(p)["kv_len"]) == [0, 36]
+
+
+def test_null_pointers_rejected_by_c_abi():
+    lib = M.load_library()
+    out = ctypes.c_void_p()
+    st = lib.mla_plan(None, 0, None, None, None, None, 1, None, None, ctypes.byref(out))
+    assert st == M.MLA_ERR_INVALID_ARGUMENT and not out.value
+    st = lib.mla_plan(ctypes.byref(M._Dims(16, 512, 64, 16, 4, SCALE)), 1, None, None, None, None, 1, None,
+                      ctypes.byref(M._Options(0, 0, 0, 0, 1)), ctypes.byref(out))
+    assert st == M.MLA_ERR_INVALID_ARGUMENT
+    assert lib.mla_plan_check(None) == M.MLA_ERR_INVALID_ARGUMENT
+    assert lib.mla_run(None, None, None, None, None, None, None) == M.MLA_ERR_INVALID_ARGUMENT
+    lib.mla_plan_destroy(None)  # no-op
+
+
+def test_host_only_plan_cannot_run():
+    p = _plan()
+    lib = M.load_library()
+    assert lib.mla_run(p.handle, None, None, None, None, None, None) == M.MLA_ERR_INVALID_ARGUMENT
+    assert lib.mla_plan_check(p.handle) == M.MLA_OK
