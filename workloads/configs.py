@@ -100,13 +100,15 @@ def make_custom(
     name: str = "custom",
     gen: Optional[torch.Generator] = None,
     pool_pages: Optional[int] = None,
+    tables_only: bool = False,
 ) -> MlaInputs:
     """Build one seeded workload from explicit per-row query and key counts.
 
     ``shared_group`` rows in a row (0 = none) name the same first ``shared_pages``
     physical pages (a shared prefix); every other page is unique to its row.
     ``pool_pages`` (if given) fixes the pool size; the pages are then drawn as a
-    random subset of it (``randperm(pool)[:needed]``).
+    random subset of it (``randperm(pool)[:needed]``).  ``tables_only`` skips the
+    random tensors (they are drawn last, so the tables are the same either way).
     """
     if gen is None:
         gen = torch.Generator().manual_seed(seed)
@@ -155,9 +157,12 @@ def make_custom(
     for n in n_pages:
         kvp.append(kvp[-1] + n)
     T = qo[-1]
-    q_nope = _randn_bf16((T, num_heads, KV_LORA_RANK), gen, std)
-    q_pe = _randn_bf16((T, num_heads, ROPE_DIM), gen, std)
-    cache = _randn_bf16((pool, page_size, LATENT), gen, std)
+    if tables_only:
+        q_nope = q_pe = cache = None
+    else:
+        q_nope = _randn_bf16((T, num_heads, KV_LORA_RANK), gen, std)
+        q_pe = _randn_bf16((T, num_heads, ROPE_DIM), gen, std)
+        cache = _randn_bf16((pool, page_size, LATENT), gen, std)
     return MlaInputs(
         name=name,
         num_heads=num_heads,
@@ -183,37 +188,36 @@ def _randint(lo: int, hi: int, n: int, gen) -> list:
     return torch.randint(lo, hi + 1, (n,), generator=gen).tolist()
 
 
-def make_config(name: str, seed: int = 0) -> MlaInputs:
+def make_config(name: str, seed: int = 0, tables_only: bool = False) -> MlaInputs:
     """One of the five named workloads (see module docstring), seeded."""
     gen = torch.Generator().manual_seed(seed)
+    kw = dict(gen=gen, name=name, tables_only=tables_only)
     if name == "tiny_decode":
-        d = make_custom([1, 1], [37, 150], 16, 16, causal=True, return_lse=True, pool_pages=32,
-                        gen=gen, name=name)
+        d = make_custom([1, 1], [37, 150], 16, 16, causal=True, return_lse=True, pool_pages=32, **kw)
         d.description = ("2 rows, q_len 1, kv lens 37 and 150, H=16, page_size 16, 13 pages "
                          "drawn from a permuted 32-page pool, lse on")
         return d
     if name == "decode_b64":
         kv = _randint(512, 8192, 64, gen)
-        d = make_custom([1] * 64, kv, 128, 64, causal=True, return_lse=False, gen=gen, name=name)
+        d = make_custom([1] * 64, kv, 128, 64, causal=True, return_lse=False, **kw)
         d.description = "64 rows, q_len 1, kv ~ U{512..8192}, H=128, page_size 64, shuffled pool, lse off"
         return d
     if name == "long_decode":
-        d = make_custom([1] * 16, [32768] * 16, 128, 64, causal=True, return_lse=True, gen=gen,
-                        name=name)
+        d = make_custom([1] * 16, [32768] * 16, 128, 64, causal=True, return_lse=True, **kw)
         d.description = "16 rows, q_len 1, kv 32768, H=128, page_size 64, lse on"
         return d
     if name == "mixed_prefill":
         kv_dec = _randint(1024, 4096, 60, gen)
         q = [1024] * 4 + [1] * 60
         kv = [2048 + 1024] * 4 + kv_dec
-        d = make_custom(q, kv, 128, 64, causal=True, return_lse=False, gen=gen, name=name)
+        d = make_custom(q, kv, 128, 64, causal=True, return_lse=False, **kw)
         d.description = ("4 prefill rows (1024 new tokens after a 2048-token prefix, causal "
                          "end-aligned) + 60 decode rows kv ~ U{1024..4096}; H=128, page_size 64")
         return d
     if name == "spec_shared_prefix":
         kv = _randint(1024, 16384, 128, gen)
         d = make_custom([4] * 128, kv, 128, 64, causal=True, return_lse=True, shared_group=8,
-                        shared_pages=16, gen=gen, name=name)
+                        shared_pages=16, **kw)
         d.description = ("128 rows, q_len 4 (causal, end-aligned), kv ~ U{1024..16384}, groups of 8 "
                          "rows share their first 1024 tokens of pages; H=128, page_size 64, lse on")
         return d
