@@ -57,7 +57,7 @@ typedef struct {
   int32_t rope_dim;     /* kpe width; must be 64                                   */
   int32_t page_size;    /* tokens per page; 16, 32, 64 or 128                      */
   int32_t num_pages;    /* pages in the cache pool (cache.shape[0]) , >= 1         */
-  float sm_scale;       /* softmax scale applied to q.k                            */
+  float sm_scale;       /* softmax scale applied to q.k; finite and > 0            */
 } mla_dims;
 
 /* Optional planning knobs; pass NULL for the defaults (all zero). */
@@ -77,6 +77,8 @@ typedef struct {
 } mla_plan_options;
 
 #define MLA_DEBUG_DROP_FIRST_KV_LOAD 1
+#define MLA_DEBUG_KERNEL_TIMING 2 /* bit 1: mla_run records CUDA events around each of its
+                                     launches (see mla_plan_kernel_times)              */
 
 /* Counts describing a plan (for callers that size buffers, and for tests). */
 typedef struct {
@@ -153,6 +155,16 @@ mla_status mla_plan_get_info(mla_plan_t plan, mla_plan_info* info);
 #define MLA_WORK_FIELDS 8
 #define MLA_MERGE_FIELDS 4
 mla_status mla_plan_describe(mla_plan_t plan, int32_t* kv_len, int32_t* work, int32_t* merge);
+
+/* Kernel durations of the plan's most recent runs, for plans made with
+ * MLA_DEBUG_KERNEL_TIMING: each mla_run records events on its stream before the
+ * attention launch, between the attention and merge launches, and after the merge.
+ * Waits for the last run, then writes up to `capacity` entries, oldest first (the plan
+ * keeps the last 256 runs): attn_ms[i] = attention kernel time, merge_ms[i] = merge
+ * kernel time (0 when the plan has no split).  *count receives the number written.
+ * Errors: INVALID_ARGUMENT (NULL, or a plan made without the flag), CUDA. */
+mla_status mla_plan_kernel_times(mla_plan_t plan, int32_t capacity, float* attn_ms, float* merge_ms,
+                                 int32_t* count);
 
 /* Wait for the plan's last run, then free everything it owns.  NULL is a no-op. */
 void mla_plan_destroy(mla_plan_t plan);

@@ -7,7 +7,7 @@ is no other implementation to fall back to.
 
 Names follow the C ABI in ``include/mla.h``: ``mla_supports``, ``mla_plan``,
 ``mla_run``, ``mla_plan_check``, ``mla_plan_get_info``, ``mla_plan_describe``,
-``mla_plan_destroy``, ``mla_status_string``.
+``mla_plan_kernel_times``, ``mla_plan_destroy``, ``mla_status_string``.
 """
 
 from __future__ import annotations
@@ -28,6 +28,7 @@ MLA_ERR_CUDA = 3
 MLA_ERR_OUT_OF_MEMORY = 4
 MLA_ERR_DEVICE_TIMEOUT = 5
 MLA_DEBUG_DROP_FIRST_KV_LOAD = 1
+MLA_DEBUG_KERNEL_TIMING = 2
 WORK_FIELDS = 8
 MERGE_FIELDS = 4
 KV_LORA_RANK = 512
@@ -40,6 +41,7 @@ EXPORTED = (
     "mla_plan_check",
     "mla_plan_get_info",
     "mla_plan_describe",
+    "mla_plan_kernel_times",
     "mla_plan_destroy",
     "mla_status_string",
 )
@@ -112,6 +114,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_plan_get_info.restype = ctypes.c_int
     lib.mla_plan_describe.argtypes = [vp, i32p, i32p, i32p]
     lib.mla_plan_describe.restype = ctypes.c_int
+    fp = ctypes.POINTER(ctypes.c_float)
+    lib.mla_plan_kernel_times.argtypes = [vp, ctypes.c_int32, fp, fp, i32p]
+    lib.mla_plan_kernel_times.restype = ctypes.c_int
     lib.mla_plan_destroy.argtypes = [vp]
     lib.mla_plan_destroy.restype = None
     lib.mla_status_string.argtypes = [ctypes.c_int]
@@ -269,6 +274,19 @@ def mla_run(plan: MlaPlan, q_nope, q_pe, cache, out=None, lse=None, return_lse: 
     if st != MLA_OK:
         raise MlaError(st, "mla_run")
     return (out, lse) if (return_lse or lse is not None) else out
+
+
+def mla_plan_kernel_times(plan: MlaPlan, capacity: int = 256):
+    """(attn_ms, merge_ms) arrays of the plan's recent runs (plans made with
+    ``debug_flags=MLA_DEBUG_KERNEL_TIMING``)."""
+    a = np.zeros(max(1, capacity), dtype=np.float32)
+    m = np.zeros(max(1, capacity), dtype=np.float32)
+    n = ctypes.c_int32(0)
+    st = load_library().mla_plan_kernel_times(plan.handle, capacity, a.ctypes.data_as(ctypes.POINTER(ctypes.c_float)),
+                                              m.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), ctypes.byref(n))
+    if st != MLA_OK:
+        raise MlaError(st, "mla_plan_kernel_times")
+    return a[: n.value], m[: n.value]
 
 
 def mla_plan_check(plan: MlaPlan) -> int:

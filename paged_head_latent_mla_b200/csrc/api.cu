@@ -33,6 +33,10 @@ struct mla_plan_s {
   float* d_ws = nullptr;  // [partials * 128 * 512] o, then [partials * 128] lse
   void* h_staging = nullptr;
   cudaEvent_t ev_last = nullptr;
+  // kernel timing ring (MLA_DEBUG_KERNEL_TIMING): 3 events per run
+  static constexpr int kRing = 256;
+  cudaEvent_t* ring = nullptr;
+  int64_t runs = 0;
 };
 
 namespace {
@@ -77,6 +81,11 @@ void free_plan(mla_plan_s* p) {
     if (p->ev_last) {
       cudaEventSynchronize(p->ev_last);
       cudaEventDestroy(p->ev_last);
+    }
+    if (p->ring) {
+      for (int i = 0; i < 3 * mla_plan_s::kRing; ++i)
+        if (p->ring[i]) cudaEventDestroy(p->ring[i]);
+      delete[] p->ring;
     }
     if (p->d_blob) cudaFree(p->d_blob);
     if (p->d_ws) cudaFree(p->d_ws);
@@ -162,6 +171,12 @@ mla_status mla_plan(const mla_dims* dims, int32_t batch, const int32_t* qo_indpt
     const size_t ws = static_cast<size_t>(p->layout.num_partials) * kTileM * (kCkv + 1) * sizeof(float);
     if (cudaMalloc(&p->d_ws, ws) != cudaSuccess) { cudaGetLastError(); free_plan(p); return MLA_ERR_OUT_OF_MEMORY; }
   }
+  if (p->opts.debug_flags & MLA_DEBUG_KERNEL_TIMING) {
+    p->ring = new (std::nothrow) cudaEvent_t[3 * mla_plan_s::kRing]();
+    if (!p->ring) { free_plan(p); return MLA_ERR_OUT_OF_MEMORY; }
+    for (int i = 0; i < 3 * mla_plan_s::kRing; ++i)
+      if (cudaEventCreate(&p->ring[i]) != cudaSuccess) { cudaGetLastError(); free_plan(p); return MLA_ERR_CUDA; }
+  }
   if (cudaEventCreateWithFlags(&p->ev_last, cudaEventDisableTiming) != cudaSuccess ||
       cudaMemcpyAsync(p->d_blob, p->h_staging, blob, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaEventRecord(p->ev_last, s) != cudaSuccess) {
@@ -200,6 +215,9 @@ mla_status mla_run(mla_plan_t p, const void* q_nope, const void* q_pe, const voi
   AttnParams ap;
   ap.work = p->d_work;
   ap.kv_indices = p->d_kv_indices;
+  ap.q_nope = q_nope;
+  ap.q_pe = q_pe;
+  ap.total_rows = static_cast<int32_t>(rows);
   ap.out = out;
   ap.lse = lse;
   ap.ws_o = p->d_ws;
@@ -211,12 +229,19 @@ mla_status mla_run(mla_plan_t p, const void* q_nope, const void* q_pe, const voi
   ap.box_rows = static_cast<int32_t>(box_rows);
   ap.timeout_ns = p->opts.wait_timeout_ns ? p->opts.wait_timeout_ns : 4000000000ull;
   ap.debug_flags = p->opts.debug_flags;
+  cudaEvent_t* ev = p->ring ? p->ring + 3 * (p->runs % mla_plan_s::kRing) : nullptr;
+  if (ev && cudaEventRecord(ev[0], s) != cudaSuccess) return MLA_ERR_CUDA;
   cudaError_t e = launch_attention(tm_q, tm_qpe, tm_kv, tm_kpe, ap, static_cast<int>(p->layout.work.size()), s);
   if (e != cudaSuccess) return MLA_ERR_CUDA;
+  if (ev && cudaEventRecord(ev[1], s) != cudaSuccess) return MLA_ERR_CUDA;
   if (!p->layout.merge.empty()) {
     MergeParams mp{p->d_merge, ap.ws_o, ap.ws_lse, ap.out, lse};
     e = launch_merge(mp, static_cast<int>(p->layout.merge.size()), s);
     if (e != cudaSuccess) return MLA_ERR_CUDA;
+  }
+  if (ev) {
+    if (cudaEventRecord(ev[2], s) != cudaSuccess) return MLA_ERR_CUDA;
+    ++p->runs;
   }
   if (cudaEventRecord(p->ev_last, s) != cudaSuccess) return MLA_ERR_CUDA;
   return MLA_OK;
@@ -257,6 +282,26 @@ mla_status mla_plan_describe(mla_plan_t p, int32_t* kv_len, int32_t* work, int32
     std::memcpy(work, p->layout.work.data(), sizeof(WorkItem) * p->layout.work.size());
   if (merge && !p->layout.merge.empty())
     std::memcpy(merge, p->layout.merge.data(), sizeof(MergeItem) * p->layout.merge.size());
+  return MLA_OK;
+}
+
+mla_status mla_plan_kernel_times(mla_plan_t p, int32_t capacity, float* attn_ms, float* merge_ms,
+                                 int32_t* count) {
+  if (!p || !p->ring || capacity < 0 || !count || (capacity > 0 && (!attn_ms || !merge_ms)))
+    return MLA_ERR_INVALID_ARGUMENT;
+  *count = 0;
+  const int64_t have = p->runs < mla_plan_s::kRing ? p->runs : mla_plan_s::kRing;
+  const int64_t n = have < capacity ? have : capacity;
+  if (n == 0) return MLA_OK;
+  if (cudaEventSynchronize(p->ring[3 * ((p->runs - 1) % mla_plan_s::kRing) + 2]) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  for (int64_t i = 0; i < n; ++i) {
+    const cudaEvent_t* ev = p->ring + 3 * ((p->runs - n + i) % mla_plan_s::kRing);
+    if (cudaEventElapsedTime(&attn_ms[i], ev[0], ev[1]) != cudaSuccess ||
+        cudaEventElapsedTime(&merge_ms[i], ev[1], ev[2]) != cudaSuccess)
+      return MLA_ERR_CUDA;
+  }
+  *count = static_cast<int32_t>(n);
   return MLA_OK;
 }
 

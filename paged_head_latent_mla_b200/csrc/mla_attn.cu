@@ -44,45 +44,63 @@ using namespace ptx;
 
 namespace attn {
 
-constexpr int kStages = 3;
-constexpr int kThreads = 192;
+#ifndef MLA_KV_STAGES
+#define MLA_KV_STAGES 4
+#endif
+#ifndef MLA_X_SLOTS
+#define MLA_X_SLOTS 1
+#endif
+constexpr int kStages = MLA_KV_STAGES;  // KV ring depth
+constexpr int kXSlots = MLA_X_SLOTS;    // exchange buffers (1 or 2)
+constexpr int kThreads = 352;  // 11 warps, roles below
+
+// Warp roles.  Warps 0..3 and 4..7 each cover the four TMEM lane quarters (a warp may
+// only touch lanes 32 * (warp % 4) .. + 31).
+constexpr int kWarpSoftmax0 = 0;   // 0..3: softmax, lazy rescale, P, epilogue
+constexpr int kWarpExchange0 = 4;  // 4..7: push our partial scores to the peer CTA
+constexpr int kWarpProducer = 8;   // TMA page gather
+constexpr int kWarpMma = 9;        // QK^T issue, TMEM allocation, zeroing past-the-end keys
+constexpr int kWarpPv = 10;        // P.V issue
+static_assert(kWarpSoftmax0 == 0 && kWarpExchange0 == 4, "quarter = warp % 4 in both groups");
 
 // Shared-memory map (offsets from a 1024-byte aligned base).
-constexpr uint32_t kQCkv = 0;              // 4 chunks x [128 rows x 128 B], 128B swizzle
-constexpr uint32_t kQKpe = 65536;          // [128 rows x 64 B], 64B swizzle
-constexpr uint32_t kKV = 73728;            // kStages stages
+constexpr uint32_t kQCkv = 0;              // 3 chunks x [128 rows x 128 B], 128B swizzle
+constexpr int kQSmemChunks = 3;            // the 4th ckv chunk and the kpe part live in TMEM
+constexpr uint32_t kKV = 49152;            // kStages stages
 constexpr uint32_t kStageBytes = 36864;    //   4 chunks x [64 keys x 128 B] + [64 x 64 B]
 constexpr uint32_t kStageKpe = 32768;
-constexpr uint32_t kX = kKV + kStages * kStageBytes;  // peer partial scores
-constexpr uint32_t kXRowBytes = 272;                  // 64 fp32 + 16 B pad (no bank conflicts)
-constexpr uint32_t kXBytes = 128 * kXRowBytes;
-constexpr uint32_t kBar = kX + kXBytes;
-constexpr uint32_t kMisc = kBar + 256;
+constexpr uint32_t kX = kKV + kStages * kStageBytes;  // the peer's partial scores
+constexpr uint32_t kXSlotBytes = 128 * 64 * 4;       // 4 quarters x 16 chunks x 32 lanes x 16 B
+constexpr uint32_t kBar = kX + kXSlots * kXSlotBytes;
+constexpr uint32_t kMisc = kBar + 512;
 constexpr uint32_t kSmemUsed = kMisc + 64;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
 // Barrier indices (8 bytes each from kBar).
-constexpr int bQFull = 0;
-constexpr int bKVFull = 1;                 // + stage
+constexpr int bQFull = 0;                   // TMA part of Q landed
+constexpr int bQTmem = 1;                   // TMEM part of Q stored (4 softmax warps)
+constexpr int bKVFull = 2;                  // + stage
 constexpr int bKVEmpty = bKVFull + kStages;
 constexpr int bSFull = bKVEmpty + kStages;  // + buffer (2)
 constexpr int bSEmpty = bSFull + 2;
 constexpr int bPFull = bSEmpty + 2;
-constexpr int bPVDone = bPFull + 2;
-constexpr int bXFull = bPVDone + 1;         // + quarter (4)
-constexpr int bXEmpty = bXFull + 4;
-constexpr int bFin = bXEmpty + 4;
-constexpr int kNumBars = bFin + 1;
-static_assert(kNumBars * 8 <= 256, "barrier area");
+constexpr int bPVDone = bPFull + 2;         // + P buffer (2): PV(j) done, j % 2
+constexpr int bXFull = bPVDone + 2;         // + slot * 4 + quarter
+constexpr int bXEmpty = bXFull + 4 * kXSlots;
+constexpr int bFin = bXEmpty + 4 * kXSlots;  // + issuer (2)
+constexpr int kNumBars = bFin + 2;
+static_assert(kNumBars * 8 <= 512, "barrier area");
 
 // TMEM columns.
 constexpr uint32_t kColO = 0;     // 256 fp32 columns: this CTA's half of O
 constexpr uint32_t kColS = 256;   // 2 x 64 fp32 columns
 constexpr uint32_t kColP = 384;   // 2 x 32 columns of packed bf16 pairs
+constexpr uint32_t kColQ = 448;   // 32 columns: ckv chunk 3 of Q (64 bf16), packed pairs
+constexpr uint32_t kColQpe = 480; // 16 columns: this CTA's 32 kpe columns of Q
 constexpr uint32_t kTmemCols = 512;
 
-constexpr uint32_t kQBytes = 65536 + 8192;
+constexpr uint32_t kQBytes = kQSmemChunks * 16384;
 constexpr float kNegInf = -__builtin_huge_valf();
 
 // Error sites (bits 8.. of the status word) for diagnosis.
@@ -97,6 +115,7 @@ enum : int32_t {
   kSiteSoftPV = 8,
   kSiteEpilogue = 9,
   kSiteTeardown = 10,
+  kSiteExchange = 11,
 };
 
 __device__ __forceinline__ void record_error(int32_t* status, int32_t site) {
@@ -105,6 +124,12 @@ __device__ __forceinline__ void record_error(int32_t* status, int32_t site) {
 
 }  // namespace attn
 
+// Pipeline per 64-key tile j (phases of every two-buffer barrier are j >> 1):
+//   producer : KV(j) -> stage j % 3                        (after PV(j - 3) freed it)
+//   QK warp  : QK(j) -> S[j % 2], as soon as KV(j) landed and S(j - 2) was read
+//   exchange : S(j) partial -> peer over DSMEM (st.async, completes the peer's x_full)
+//   softmax  : S(j) = ours + peer's; mask, online softmax, P(j) -> P[j % 2]
+//   PV warp  : PV(j): O += P[j % 2] . V(stage j % 3), as soon as P(j) is written
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     mla_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qpe,
                     const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_kpe,
@@ -126,30 +151,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(bar(bQFull), 1);
+    mbar_init(bar(bQTmem), 4);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(bKVFull + s), 1);
       mbar_init(bar(bKVEmpty + s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(bSFull + b), 1);
-      mbar_init(bar(bSEmpty + b), 4);
+      mbar_init(bar(bSEmpty + b), 8);  // softmax and exchange warps both read S
       mbar_init(bar(bPFull + b), 4);
+      mbar_init(bar(bPVDone + b), 1);
     }
-    mbar_init(bar(bPVDone), 1);
-    for (int q = 0; q < 4; ++q) {
-      mbar_init(bar(bXFull + q), 32);
-      mbar_init(bar(bXEmpty + q), 32);
+    for (int i = 0; i < 4 * kXSlots; ++i) {
+      mbar_init(bar(bXFull + i), 1);   // our expect_tx + the peer's 8 KB of st.async
+      mbar_init(bar(bXEmpty + i), 1);  // the peer drained the 8 KB we pushed
     }
     mbar_init(bar(bFin), 1);
+    mbar_init(bar(bFin + 1), 1);
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == kWarpProducer && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_qpe);
     tma_prefetch_desc(&tm_kv);
     tma_prefetch_desc(&tm_kpe);
   }
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tmem_alloc(smem_addr(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
@@ -162,46 +189,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint64_t TO = p.timeout_ns;
 
-  if (warp == 0) {
+  // Bounded wait shared by every role: all lanes poll, the warp agrees, lane 0 records.
+  auto wait_warp = [&](uint32_t b, uint32_t parity, int32_t site, bool cluster_scope) -> bool {
+    bool good = cluster_scope ? mbar_wait<true>(b, parity, TO, abort_flag) : mbar_wait(b, parity, TO, abort_flag);
+    good = __all_sync(0xffffffffu, good);
+    if (!good && lane == 0) {
+      record_error(p.status, site);
+      *abort_flag = 1;
+    }
+    return good;
+  };
+
+  if (warp == kWarpProducer) {
     // ------------------------------------------------------------------ TMA producer
     if (ntiles > 0) {
       if (lane == 0) {
         mbar_arrive_expect_tx(bar(bQFull), kQBytes);
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < kQSmemChunks; ++c)
           tma_load_2d(sb + kQCkv + c * 16384, &tm_q, bar(bQFull), 256 * rank + 64 * c, w.q_row0);
-        tma_load_2d(sb + kQKpe, &tm_qpe, bar(bQFull), 32 * rank, w.q_row0);
       }
       const int P = p.page_size, BR = p.box_rows, nbox = kTileN / BR;
       const int last_page = (w.kv_len + P - 1) / P - 1;
-      // physical start row of box `lane` of tile j (lanes >= nbox unused)
-      auto box_row = [&](int j) -> int {
-        int rs = 0;
-        if (lane < nbox) {
-          const int key0 = w.key_begin + kTileN * j + lane * BR;
-          const int lp = min(key0 / P, last_page);
-          rs = __ldg(p.kv_indices + w.page_base + lp) * P + (key0 % P);
+      // Page ids are read 32 at a time (lane i holds logical page win + i) so that no
+      // dependent global load sits between a free stage and its TMA issue.
+      int win = -64, win_id = 0;
+      auto page_of = [&](int lp) -> int {
+        lp = min(lp, last_page);
+        if (lp - win < 0 || lp - win >= 32) {  // warp-uniform
+          win = lp;
+          win_id = (win + lane <= last_page) ? __ldg(p.kv_indices + w.page_base + win + lane) : 0;
         }
-        return rs;
+        return __shfl_sync(0xffffffffu, win_id, lp - win);
       };
-      int last_issued[kStages] = {-1, -1, -1};
-      int rs_next = box_row(0);
+      int last_issued[kStages];
+#pragma unroll
+      for (int s2 = 0; s2 < kStages; ++s2) last_issued[s2] = -1;
       for (int j = 0; j < ntiles; ++j) {
         const int st = j % kStages;
-        const int rs = rs_next;
-        if (j + 1 < ntiles) rs_next = box_row(j + 1);
-        if (j >= kStages) {
-          bool ok = mbar_wait(bar(bKVEmpty + st), ((j / kStages) - 1) & 1, TO, abort_flag);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) {
-            if (lane == 0) { record_error(p.status, kSiteProducer); *abort_flag = 1; }
-            break;
-          }
-        }
+        if (j >= kStages && !wait_warp(bar(bKVEmpty + st), ((j / kStages) - 1) & 1, kSiteProducer, false)) break;
         if ((p.debug_flags & MLA_DEBUG_DROP_FIRST_KV_LOAD) && j == 0) continue;
         const uint32_t dst = sb + kKV + st * kStageBytes;
         if (lane == 0) mbar_arrive_expect_tx(bar(bKVFull + st), kStageBytes);
         for (int b = 0; b < nbox; ++b) {
-          const int row = __shfl_sync(0xffffffffu, rs, b);
+          const int key0 = w.key_begin + kTileN * j + b * BR;
+          const int row = page_of(key0 / P) * P + (key0 % P);
           if (lane == 0) {
             for (int c = 0; c < 4; ++c)
               tma_load_2d(dst + c * 8192 + b * BR * 128, &tm_kv, bar(bKVFull + st), 256 * rank + 64 * c, row);
@@ -219,36 +250,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
             record_error(p.status, kSiteTeardown);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
     if (ntiles > 0) {
       const uint32_t id_qk = idesc_bf16_f32(128, 64, false, false);
-      const uint32_t id_pv = idesc_bf16_f32(128, 256, false, true);
-      bool ok = mbar_wait(bar(bQFull), 0, TO, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok && lane == 0) { record_error(p.status, kSiteMmaQ); *abort_flag = 1; }
-      tc_fence_after();
-      auto issue_pv = [&](int j) {
-        const uint32_t kv = sb + kKV + (j % kStages) * kStageBytes;
-        const uint32_t pcol = tmem + kColP + 32 * (j & 1);
-        for (int s = 0; s < 4; ++s) {
-          const uint64_t bd = smem_desc(kv + s * 2048, 8192, 1024, 2);
-          mma_ts(tmem + kColO, pcol + 8 * s, bd, id_pv, (j > 0 || s > 0) ? 1u : 0u);
-        }
-        mma_commit(bar(bKVEmpty + (j % kStages)));
-        mma_commit(bar(bPVDone));
-      };
-      int j = 0;
-      for (; ok && j < ntiles; ++j) {
+      // QK(j): wait for KV(j) and for both readers of S(j - 2) to be done with S[j % 2].
+      auto issue_qk = [&](int j) -> bool {
         const int st = j % kStages, b2 = j & 1;
-        ok = mbar_wait(bar(bKVFull + st), (j / kStages) & 1, TO, abort_flag);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) { if (lane == 0) { record_error(p.status, kSiteMmaKV); *abort_flag = 1; } break; }
-        if (j >= 2) {
-          ok = mbar_wait(bar(bSEmpty + b2), ((j >> 1) - 1) & 1, TO, abort_flag);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) { if (lane == 0) { record_error(p.status, kSiteMmaS); *abort_flag = 1; } break; }
-        }
+        if (!wait_warp(bar(bKVFull + st), (j / kStages) & 1, kSiteMmaKV, false)) return false;
+        if (j >= 2 && !wait_warp(bar(bSEmpty + b2), ((j >> 1) - 1) & 1, kSiteMmaS, false)) return false;
         tc_fence_after();
         const uint32_t kv = sb + kKV + st * kStageBytes;
         // Keys at or past the row's end hold whatever the page's unused slots contain;
@@ -260,56 +270,95 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
           for (int i = lane; i < 4 * n16; i += 32) {
             const int c = i / n16, k = i % n16;
-            float4* dst = reinterpret_cast<float4*>(smem + kKV + st * kStageBytes + c * 8192 +
-                                                    first_bad * 128 + k * 16);
-            *dst = z;
+            *reinterpret_cast<float4*>(smem + kKV + st * kStageBytes + c * 8192 + first_bad * 128 + k * 16) = z;
           }
           fence_proxy_async_smem();
           __syncwarp();
         }
         if (lane == 0) {
           const uint32_t scol = tmem + kColS + 64 * b2;
-          for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < kQSmemChunks; ++c)
             for (int s = 0; s < 4; ++s) {
               const uint64_t ad = smem_desc(sb + kQCkv + c * 16384 + s * 32, 16, 1024, 2);
               const uint64_t bd = smem_desc(kv + c * 8192 + s * 32, 16, 1024, 2);
               mma_ss(scol, ad, bd, id_qk, (c | s) ? 1u : 0u);
             }
-          for (int s = 0; s < 2; ++s) {
-            const uint64_t ad = smem_desc(sb + kQKpe + s * 32, 16, 512, 4);
+          for (int s = 0; s < 4; ++s) {  // ckv chunk 3: A from TMEM
+            const uint64_t bd = smem_desc(kv + 3 * 8192 + s * 32, 16, 1024, 2);
+            mma_ts(scol, tmem + kColQ + 8 * s, bd, id_qk, 1u);
+          }
+          for (int s = 0; s < 2; ++s) {  // kpe: A from TMEM
             const uint64_t bd = smem_desc(kv + kStageKpe + s * 32, 16, 512, 4);
-            mma_ss(scol, ad, bd, id_qk, 1u);
+            mma_ts(scol, tmem + kColQpe + 8 * s, bd, id_qk, 1u);
           }
           mma_commit(bar(bSFull + b2));
         }
         __syncwarp();
-        if (j >= 1) {
-          ok = mbar_wait(bar(bPFull + ((j - 1) & 1)), ((j - 1) >> 1) & 1, TO, abort_flag);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) { if (lane == 0) { record_error(p.status, kSiteMmaP); *abort_flag = 1; } break; }
-          tc_fence_after();
-          if (lane == 0) issue_pv(j - 1);
-          __syncwarp();
-        }
-      }
-      if (ok) {
-        const int jl = ntiles - 1;
-        ok = mbar_wait(bar(bPFull + (jl & 1)), (jl >> 1) & 1, TO, abort_flag);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) {
-          if (lane == 0) { record_error(p.status, kSiteMmaP); *abort_flag = 1; }
-        } else {
-          tc_fence_after();
-          if (lane == 0) issue_pv(jl);
-          __syncwarp();
-        }
-      }
+        return true;
+      };
+      bool ok = wait_warp(bar(bQFull), 0, kSiteMmaQ, false) && wait_warp(bar(bQTmem), 0, kSiteMmaQ, false);
+      tc_fence_after();
+      for (int j = 0; ok && j < ntiles; ++j) ok = issue_qk(j);
       // Every MMA this thread issued must retire before TMEM is released.
       if (lane == 0) {
         mma_commit(bar(bFin));
         if (!mbar_wait(bar(bFin), 0, TO, abort_flag)) record_error(p.status, kSiteTeardown);
       }
       __syncwarp();
+    }
+  } else if (warp == kWarpPv) {
+    // ------------------------------------------------------------------ P.V issuer
+    if (ntiles > 0) {
+      const uint32_t id_pv = idesc_bf16_f32(128, 256, false, true);
+      for (int j = 0; j < ntiles; ++j) {
+        if (!wait_warp(bar(bPFull + (j & 1)), (j >> 1) & 1, kSiteMmaP, false)) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t kv = sb + kKV + (j % kStages) * kStageBytes;
+          const uint32_t pcol = tmem + kColP + 32 * (j & 1);
+          for (int s = 0; s < 4; ++s) {
+            const uint64_t bd = smem_desc(kv + s * 2048, 8192, 1024, 2);
+            mma_ts(tmem + kColO, pcol + 8 * s, bd, id_pv, (j > 0 || s > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(bKVEmpty + (j % kStages)));
+          mma_commit(bar(bPVDone + (j & 1)));
+        }
+        __syncwarp();
+      }
+      if (lane == 0) {
+        mma_commit(bar(bFin + 1));
+        if (!mbar_wait(bar(bFin + 1), 0, TO, abort_flag)) record_error(p.status, kSiteTeardown);
+      }
+      __syncwarp();
+    }
+  } else if (warp >= kWarpExchange0) {
+    // ------------------------------------------------------------------ score exchange
+    // Partial S(j) (our 288 of the 576 contraction columns) goes to the peer, laid out
+    // chunk-major per lane quarter: 16-byte chunk c of row (32q + lane) sits at
+    // q * 8 KB + (c * 32 + lane) * 16, so one warp store covers 512 contiguous bytes.
+    const int q = warp & 3;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    const uint32_t xq_peer = map_to_cta(sb + kX + q * 8192 + lane * 16, peer);
+    const uint32_t xfull_peer = map_to_cta(bar(bXFull + q), peer);
+    for (int j = 0; j < ntiles; ++j) {
+      const int b2 = j & 1;
+      if (!wait_warp(bar(bSFull + b2), (j >> 1) & 1, kSiteExchange, false)) break;
+      tc_fence_after();
+      uint32_t sr[64];
+      tmem_ld32(trow + kColS + 64 * b2, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(trow + kColS + 64 * b2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(bSEmpty + b2));
+      // the peer must have drained our slot (it held tile j - kXSlots)
+      const int xs = j % kXSlots, xph = j / kXSlots;
+      if (j >= kXSlots && !wait_warp(bar(bXEmpty + 4 * xs + q), (xph - 1) & 1, kSiteExchange, true)) break;
+      const uint32_t dst = xq_peer + xs * kXSlotBytes;
+      const uint32_t xbar = xfull_peer + 8u * (4 * xs);
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        st_async_v4(dst + c * 512, sr[4 * c], sr[4 * c + 1], sr[4 * c + 2], sr[4 * c + 3], xbar);
     }
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
@@ -320,16 +369,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     vis = max(0, min(vis, w.kv_len));
     if (r >= w.n_rows) vis = 0;
     const int lim = min(vis, w.key_end);  // keys < lim are visible in this chunk
-    const uint32_t xrow = sb + kX + r * kXRowBytes;
-    const uint32_t xrow_peer = map_to_cta(xrow, peer);
-    const float* xrow_ptr = reinterpret_cast<const float*>(smem + kX + r * kXRowBytes);
+    const float* xq_ptr = reinterpret_cast<const float*>(smem + kX + q * 8192 + lane * 16);
+    const float scale = p.scale_log2;  // > 0 (the planner rejects other scales)
     float m_run = kNegInf, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
+
+    // --- the TMEM part of Q: ckv columns [256r + 192, 256r + 256) and kpe columns
+    // [32r, 32r + 32) of this row, as packed bf16 pairs (even element in the low half)
+    if (ntiles > 0) {
+      uint32_t qa[32], qb[16];
+      if (r < w.n_rows) {
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q_nope) +
+                                                          static_cast<size_t>(w.q_row0 + r) * kCkv + 256 * rank + 192);
+        const uint4* srp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q_pe) +
+                                                          static_cast<size_t>(w.q_row0 + r) * kRope + 32 * rank);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 v = __ldg(src + i);
+          qa[4 * i] = v.x; qa[4 * i + 1] = v.y; qa[4 * i + 2] = v.z; qa[4 * i + 3] = v.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 v = __ldg(srp + i);
+          qb[4 * i] = v.x; qb[4 * i + 1] = v.y; qb[4 * i + 2] = v.z; qb[4 * i + 3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) qa[i] = 0u;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) qb[i] = 0u;
+      }
+      tmem_st32(trow + kColQ, qa);
+      tmem_st16(trow + kColQpe, qb);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(bQTmem));
+    }
+
+    for (int j = 0; ok && j < ntiles; ++j) {
       const int b2 = j & 1;
-      ok = mbar_wait(bar(bSFull + b2), (j >> 1) & 1, TO, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) { if (lane == 0) { record_error(p.status, kSiteSoftS); *abort_flag = 1; } break; }
+      if (!(ok = wait_warp(bar(bSFull + b2), (j >> 1) & 1, kSiteSoftS, false))) break;
+      const int xsl = j % kXSlots, xph = j / kXSlots;
+      const uint32_t xfull = bar(bXFull + 4 * xsl + q);
+      if (lane == 0) mbar_arrive_expect_tx(xfull, 8192);
       tc_fence_after();
       uint32_t sr[64];
       tmem_ld32(trow + kColS + 64 * b2, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
@@ -338,40 +421,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(bSEmpty + b2));
-
-      // --- exchange partial scores with the peer CTA
-      if (j >= 1) {
-        ok = mbar_wait<true>(bar(bXEmpty + q), (j - 1) & 1, TO, abort_flag);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) { if (lane == 0) { record_error(p.status, kSiteSoftX); *abort_flag = 1; } break; }
-      }
-#pragma unroll
-      for (int c = 0; c < 16; ++c)
-        st_cluster_v4(xrow_peer + 16 * c, __uint_as_float(sr[4 * c]), __uint_as_float(sr[4 * c + 1]),
-                      __uint_as_float(sr[4 * c + 2]), __uint_as_float(sr[4 * c + 3]));
-      mbar_arrive_remote(bar(bXFull + q), peer);
-      ok = mbar_wait<true>(bar(bXFull + q), j & 1, TO, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) { if (lane == 0) { record_error(p.status, kSiteSoftX); *abort_flag = 1; } break; }
+      if (!(ok = wait_warp(xfull, xph & 1, kSiteSoftX, true))) break;
+      // --- raw S(j) = our partial + the peer's (fp32 addition commutes: the pair holds
+      // bit-identical scores)
+      const float* xs = xq_ptr + xsl * (kXSlotBytes / 4);
       float t[64];
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
-        const float4 x = *reinterpret_cast<const float4*>(xrow_ptr + 4 * c);
+        const float4 x = *reinterpret_cast<const float4*>(xs + c * 128);
         t[4 * c + 0] = __uint_as_float(sr[4 * c + 0]) + x.x;
         t[4 * c + 1] = __uint_as_float(sr[4 * c + 1]) + x.y;
         t[4 * c + 2] = __uint_as_float(sr[4 * c + 2]) + x.z;
         t[4 * c + 3] = __uint_as_float(sr[4 * c + 3]) + x.w;
       }
-      mbar_arrive_remote(bar(bXEmpty + q), peer);
+      // Every lane has consumed its loaded values (the sums above), so the slot can be
+      // handed back with a relaxed arrive.
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote_relaxed(bar(bXEmpty + 4 * xsl + q), peer);
 
-      // --- mask, running max (log2 domain), lazy rescale
+      // --- mask (partial tiles only), running max in the log2 domain, lazy rescale
       const int nvalid = lim - (w.key_begin + kTileN * j);
-      float mt = kNegInf;
+      if (__any_sync(0xffffffffu, nvalid < kTileN)) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        t[c] = (c < nvalid) ? t[c] * p.scale_log2 : kNegInf;
-        mt = fmaxf(mt, t[c]);
+        for (int c = 0; c < 64; ++c) t[c] = (c < nvalid) ? t[c] : kNegInf;
       }
+      float mx[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(t[i], t[i + 8]);
+#pragma unroll
+      for (int c = 16; c < 64; c += 8)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], t[c + i]);
+      const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      const float mt = mraw * scale;  // scale > 0 keeps the order; -inf stays -inf
       // Keep the old reference max unless the new one exceeds it by more than 8 (a
       // factor of 256 in the weights); then rescale the running sum and output row.
       const bool bump = mt > m_run + 8.f;
@@ -384,9 +467,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       }
       const bool resc = bump && j > 0 && m_old != kNegInf;
       if (__any_sync(0xffffffffu, resc)) {
-        ok = mbar_wait(bar(bPVDone), (j - 1) & 1, TO, abort_flag);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) { if (lane == 0) { record_error(p.status, kSiteSoftPV); *abort_flag = 1; } break; }
+        // every PV so far (the last is PV(j - 1)) must have landed in O
+        if (!(ok = wait_warp(bar(bPVDone + ((j - 1) & 1)), ((j - 1) >> 1) & 1, kSiteSoftPV, false))) break;
         tc_fence_after();
         const float a = resc ? alpha : 1.f;
         for (int cc = 0; cc < 256; cc += 32) {
@@ -395,26 +477,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * a);
-          tmem_st16(trow + kColO + cc, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
-          tmem_st16(trow + kColO + cc + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
+          tmem_st32(trow + kColO + cc, o);
         }
         tmem_wait_st();
       }
 
-      // --- P = exp2(t - m) into TMEM as bf16; the running sum takes the fp32 values
+      // --- P = exp2(s * scale - m) as bf16 (fp32 running sum); P[j % 2] was last read
+      // by PV(j - 2)
       const float msub = (m_run == kNegInf) ? 0.f : m_run;
       uint32_t pk[32];
-      float lsum = 0.f;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        const float p0 = ex2_approx(t[2 * c] - msub);
-        const float p1 = ex2_approx(t[2 * c + 1] - msub);
+        const float p0 = ex2_approx(fmaf(t[2 * c], scale, -msub));
+        const float p1 = ex2_approx(fmaf(t[2 * c + 1], scale, -msub));
         pk[c] = pack_bf16x2(p0, p1);
-        lsum += p0 + p1;
+        ls[c & 3] += p0 + p1;
       }
-      l_run += lsum;
-      tmem_st16(trow + kColP + 32 * b2, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-      tmem_st16(trow + kColP + 32 * b2 + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+      l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      if (j >= 2 && !(ok = wait_warp(bar(bPVDone + b2), ((j >> 1) - 1) & 1, kSiteSoftPV, false))) break;
+      tc_fence_after();
+      tmem_st32(trow + kColP + 32 * b2, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -428,14 +511,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       const float lse_nat = has ? (m_run + __log2f(l_run)) * 0.69314718055994531f : kNegInf;
       const bool row_ok = r < w.n_rows;
       if (ntiles > 0) {
-        ok = mbar_wait(bar(bPVDone), (ntiles - 1) & 1, TO, abort_flag);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok && lane == 0) { record_error(p.status, kSiteEpilogue); *abort_flag = 1; }
+        ok = wait_warp(bar(bPVDone + ((ntiles - 1) & 1)), ((ntiles - 1) >> 1) & 1, kSiteEpilogue, false);
         tc_fence_after();
       }
       if (ok) {
         if (w.partial < 0) {
-          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + static_cast<size_t>(w.q_row0 + r) * kCkv + 256 * rank;
+          __nv_bfloat16* dst =
+              static_cast<__nv_bfloat16*>(p.out) + static_cast<size_t>(w.q_row0 + r) * kCkv + 256 * rank;
           for (int cc = 0; cc < 256; cc += 32) {
             uint32_t o[32];
             if (ntiles > 0) {
@@ -485,7 +567,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   // ------------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -498,9 +580,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
 // M = max_i lse_i, out = sum_i e^{lse_i - M} o_i / sum_i e^{lse_i - M},
 // lse = M + ln sum_i e^{lse_i - M} (FlashInferMLAManager.run: merging key segments).
 __global__ void __launch_bounds__(256) mla_merge_kernel(const MergeParams p) {
-  const MergeItem m = p.merge[blockIdx.x];
+  // 16 blocks per split query tile, 8 rows (one per warp) per block.
+  const MergeItem m = p.merge[blockIdx.x >> 4];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int r = warp; r < m.n_rows; r += 8) {
+  const int r = ((blockIdx.x & 15) << 3) + warp;
+  if (r < m.n_rows) {
     float M = -__int_as_float(0x7f800000);
     for (int i = 0; i < m.n_partials; ++i)
       M = fmaxf(M, p.ws_lse[static_cast<size_t>(m.first_partial + i) * kTileM + r]);
@@ -556,7 +640,7 @@ cudaError_t launch_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_qpe,
 }
 
 cudaError_t launch_merge(const MergeParams& p, int num_merge, cudaStream_t stream) {
-  mla_merge_kernel<<<num_merge, 256, 0, stream>>>(p);
+  mla_merge_kernel<<<num_merge * 16, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

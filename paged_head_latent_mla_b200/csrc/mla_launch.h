@@ -13,6 +13,9 @@ namespace mla {
 struct AttnParams {
   const WorkItem* work;
   const int32_t* kv_indices;
+  const void* q_nope;  // bf16 [T*H, 512]
+  const void* q_pe;    // bf16 [T*H, 64]
+  int32_t total_rows;  // T*H
   void* out;       // bf16 [T*H, 512]
   float* lse;      // fp32 [T*H] or nullptr
   float* ws_o;     // fp32 [partials, 128, 512]

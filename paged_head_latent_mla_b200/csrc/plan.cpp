@@ -89,7 +89,8 @@ mla_status build_layout(const mla_dims& d, int32_t batch, const int32_t* qo_indp
   if (!out) return MLA_ERR_INVALID_ARGUMENT;
   if (!shape_supported(d.kv_lora_rank, d.rope_dim, d.num_heads, d.page_size))
     return MLA_ERR_UNSUPPORTED;
-  if (batch < 0 || d.num_pages < 1 || !std::isfinite(d.sm_scale)) return MLA_ERR_INVALID_ARGUMENT;
+  if (batch < 0 || d.num_pages < 1 || !std::isfinite(d.sm_scale) || !(d.sm_scale > 0.f))
+    return MLA_ERR_INVALID_ARGUMENT;
   if (!qo_indptr || !kv_indptr || (batch > 0 && !last_page_len)) return MLA_ERR_INVALID_ARGUMENT;
   if (split_keys > 0 && split_keys % kTileN != 0) return MLA_ERR_INVALID_ARGUMENT;
   const int32_t H = d.num_heads, P = d.page_size;
