@@ -166,6 +166,40 @@ mla_status mla_plan_describe(mla_plan_t plan, int32_t* kv_len, int32_t* work, in
 mla_status mla_plan_kernel_times(mla_plan_t plan, int32_t capacity, float* attn_ms, float* merge_ms,
                                  int32_t* count);
 
+/* Plan and run one step without allocating any memory (no paper counterpart: this is a
+ * library-level entry point, not part of the method).
+ *
+ * For callers that cannot allocate when they run attention: serving processes whose
+ * memory manager has handed all of HBM to its own pools and forbids other allocations,
+ * plug-in hosts that give the library no allocator, and latency-critical loops where a
+ * cudaMalloc/cudaFree could synchronise the device.  mla_plan allocates; this call does
+ * not (no cudaMalloc, cudaFree or pinned allocation, and no heap use while planning).
+ *
+ * Arguments are those of mla_plan (host tables, copied during the call) followed by
+ * those of mla_run (device tensors, same layouts and alignment rules).  Planning uses a
+ * fixed split rule instead of mla_plan's balancing search, so the split points may
+ * differ from mla_run's; results agree within floating-point tolerance.
+ *
+ * All device scratch (status word, work list, page-table copy, split-KV partials) lives
+ * in one 16 MiB array compiled into the library; every GPU that loads the library holds
+ * it until the process exits.  Limits: kv_indptr[batch] <= 524288 page ids and at most
+ * 16384 query tiles (a tile is 128 / H tokens of one row); larger steps return
+ * MLA_ERR_INVALID_ARGUMENT.  Long key ranges are split only while the array has room
+ * for their partial results (at least 32 tiles' worth); the rest run unsplit.
+ *
+ * The first call on a device looks up the array's device address (and the SM count)
+ * with that device current; make that first call before any stream capture.  Every call
+ * shares the one array (and static host buffers), so calls must not overlap, on the host
+ * or on the GPU: issue them from one thread, on one stream, or synchronise in between.
+ * In-kernel wait timeouts are recorded in the array's status word, which is not
+ * reported back; use mla_plan/mla_run/mla_plan_check where that matters.
+ * Errors: INVALID_ARGUMENT (bad tables or pointers, or beyond the limits above),
+ * UNSUPPORTED (shape), CUDA. */
+mla_status mla_run_noalloc(const mla_dims* dims, int32_t batch, const int32_t* qo_indptr,
+                           const int32_t* kv_indptr, const int32_t* kv_indices,
+                           const int32_t* last_page_len, int32_t causal, const void* q_nope,
+                           const void* q_pe, const void* cache, void* out, float* lse, void* stream);
+
 /* Wait for the plan's last run, then free everything it owns.  NULL is a no-op. */
 void mla_plan_destroy(mla_plan_t plan);
 

@@ -7,7 +7,8 @@ is no other implementation to fall back to.
 
 Names follow the C ABI in ``include/mla.h``: ``mla_supports``, ``mla_plan``,
 ``mla_run``, ``mla_plan_check``, ``mla_plan_get_info``, ``mla_plan_describe``,
-``mla_plan_kernel_times``, ``mla_plan_destroy``, ``mla_status_string``.
+``mla_plan_kernel_times``, ``mla_run_noalloc``, ``mla_plan_destroy``,
+``mla_status_string``.
 """
 
 from __future__ import annotations
@@ -42,6 +43,7 @@ EXPORTED = (
     "mla_plan_get_info",
     "mla_plan_describe",
     "mla_plan_kernel_times",
+    "mla_run_noalloc",
     "mla_plan_destroy",
     "mla_status_string",
 )
@@ -117,6 +119,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     fp = ctypes.POINTER(ctypes.c_float)
     lib.mla_plan_kernel_times.argtypes = [vp, ctypes.c_int32, fp, fp, i32p]
     lib.mla_plan_kernel_times.restype = ctypes.c_int
+    lib.mla_run_noalloc.argtypes = [ctypes.POINTER(_Dims), ctypes.c_int32, i32p, i32p, i32p, i32p, ctypes.c_int32,
+                                    vp, vp, vp, vp, vp, vp]
+    lib.mla_run_noalloc.restype = ctypes.c_int
     lib.mla_plan_destroy.argtypes = [vp]
     lib.mla_plan_destroy.restype = None
     lib.mla_status_string.argtypes = [ctypes.c_int]
@@ -287,6 +292,42 @@ def mla_plan_kernel_times(plan: MlaPlan, capacity: int = 256):
     if st != MLA_OK:
         raise MlaError(st, "mla_plan_kernel_times")
     return a[: n.value], m[: n.value]
+
+
+def mla_run_noalloc(qo_indptr, kv_indptr, kv_indices, last_page_len, q_nope, q_pe, cache, out, lse=None, *,
+                    num_heads: int, page_size: int, num_pages: int, sm_scale: float, causal: bool = True,
+                    kv_lora_rank: int = KV_LORA_RANK, rope_dim: int = ROPE_DIM, stream=None) -> None:
+    """Plan and run one step without allocating (``mla_run_noalloc``): for callers that
+    may not allocate device memory when attention runs.  ``out`` (and ``lse`` if given)
+    must be preallocated by the caller; host tables as for ``mla_plan``.  Calls share
+    one fixed device scratch array, so they must not overlap."""
+    import torch
+
+    qo = _i32(qo_indptr)
+    kvp = _i32(kv_indptr)
+    kvi = _i32(kv_indices)
+    last = _i32(last_page_len)
+    batch = len(qo) - 1
+    if batch < 0 or len(kvp) != batch + 1 or len(last) != batch or len(kvi) < int(kvp[-1]):
+        raise MlaError(MLA_ERR_INVALID_ARGUMENT, "mla_run_noalloc: table lengths")
+    T = int(qo[-1])
+    _check_dev_tensor(q_nope, "q_nope", torch.bfloat16, (T, num_heads, kv_lora_rank))
+    _check_dev_tensor(q_pe, "q_pe", torch.bfloat16, (T, num_heads, rope_dim))
+    _check_dev_tensor(cache, "cache", torch.bfloat16, tuple(cache.shape))
+    _check_dev_tensor(out, "out", torch.bfloat16, (T, num_heads, kv_lora_rank))
+    if lse is not None:
+        _check_dev_tensor(lse, "lse", torch.float32, (T, num_heads))
+    if stream is None:
+        stream = torch.cuda.current_stream(q_nope.device).cuda_stream
+    dims = _Dims(num_heads, kv_lora_rank, rope_dim, page_size, num_pages, sm_scale)
+    kvi_arr = kvi if len(kvi) else np.zeros(1, dtype=np.int32)
+    st = load_library().mla_run_noalloc(
+        ctypes.byref(dims), batch, _ptr(qo), _ptr(kvp), _ptr(kvi_arr), _ptr(last), 1 if causal else 0,
+        ctypes.c_void_p(q_nope.data_ptr()), ctypes.c_void_p(q_pe.data_ptr()), ctypes.c_void_p(cache.data_ptr()),
+        ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(lse.data_ptr() if lse is not None else 0),
+        ctypes.c_void_p(stream or 0))
+    if st != MLA_OK:
+        raise MlaError(st, "mla_run_noalloc")
 
 
 def mla_plan_check(plan: MlaPlan) -> int:

@@ -1,0 +1,264 @@
+// mla_run_noalloc: the attention call for callers that must not allocate memory.
+//
+// Some callers cannot call cudaMalloc at the point where they run attention: serving
+// processes whose memory manager has already handed all of HBM to its own pools (a KV
+// page pool, an activation arena) and forbids any other allocation; plug-in hosts that
+// own device memory and give a library no allocator; latency-critical loops where a
+// cudaMalloc or cudaFree could synchronise the device.  mla_plan allocates (work lists,
+// page-table copy, split-KV workspace, pinned staging), so those callers use this entry
+// point instead: it plans on the host without touching the heap, and every piece of
+// device scratch it needs (status word, work list, merge list, page-table copy and the
+// split-KV partial results) lives in one array compiled into the library.
+//
+// The array is a file-scope __device__ variable: every GPU that loads the library
+// holds kScratchBytes of it until the process exits.  Host code may not use the
+// array's name as a device address (it is a host-side stand-in), so the device address
+// is looked up once per device with cudaGetSymbolAddress, with that device current.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <limits>
+#include <mutex>
+
+#include "mla_internal.h"
+#include "mla_launch.h"
+
+namespace {
+
+using namespace mla;
+
+// Fixed scratch budget and its layout.
+constexpr size_t kScratchBytes = size_t(16) << 20;  // 16 MiB per device
+constexpr int kMaxWork = 16384;                     // work items
+constexpr int kMaxMerge = 4096;                     // split query tiles
+constexpr int kMaxPageIds = 1 << 19;                // kv_indptr[batch]
+constexpr size_t kOffStatus = 0;
+constexpr size_t kOffWork = 256;
+constexpr size_t kOffMerge = kOffWork + sizeof(WorkItem) * kMaxWork;
+constexpr size_t kOffPages = kOffMerge + sizeof(MergeItem) * kMaxMerge;
+constexpr size_t kOffPartials = (kOffPages + sizeof(int32_t) * kMaxPageIds + 255) / 256 * 256;
+constexpr size_t kPartialBytes = size_t(kTileM) * (kCkv + 1) * sizeof(float);  // o + lse of one tile
+constexpr int kMaxPartials = static_cast<int>((kScratchBytes - kOffPartials) / kPartialBytes);
+static_assert(kMaxPartials >= 32, "scratch too small for useful splitting");
+
+// Host-side planning buffers: static, so planning never touches the heap.  Calls that
+// overlap on the host would race on these, like they race on the device array.
+WorkItem g_work[kMaxWork];
+MergeItem g_merge[kMaxMerge];
+
+struct DeviceScratch {
+  unsigned char* ptr = nullptr;
+  int num_sms = 0;
+};
+constexpr int kMaxDevices = 64;
+DeviceScratch g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool encode_2d(EncodeTiledFn enc, CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+               uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Validate the tables and cut the work into g_work / g_merge without allocating.
+// Long key ranges are split into chunks of about (total tiles / SM pairs) tiles while
+// partial slots remain in the scratch array; the rest run unsplit.
+mla_status plan_fixed(const mla_dims& d, int32_t batch, const int32_t* qo, const int32_t* kvp,
+                      const int32_t* kvi, const int32_t* last, bool causal, int num_sms, int* n_work,
+                      int* n_merge, int* n_partials, int32_t* total_tokens) {
+  if (!shape_supported(d.kv_lora_rank, d.rope_dim, d.num_heads, d.page_size)) return MLA_ERR_UNSUPPORTED;
+  if (batch < 0 || d.num_pages < 1 || !std::isfinite(d.sm_scale) || !(d.sm_scale > 0.f))
+    return MLA_ERR_INVALID_ARGUMENT;
+  if (!qo || !kvp || (batch > 0 && !last)) return MLA_ERR_INVALID_ARGUMENT;
+  const int32_t H = d.num_heads, P = d.page_size;
+  if (int64_t(d.num_pages) * P > std::numeric_limits<int32_t>::max()) return MLA_ERR_INVALID_ARGUMENT;
+  if (qo[0] != 0 || kvp[0] != 0) return MLA_ERR_INVALID_ARGUMENT;
+  for (int32_t b = 0; b < batch; ++b)
+    if (qo[b + 1] < qo[b] || kvp[b + 1] < kvp[b]) return MLA_ERR_INVALID_ARGUMENT;
+  const int64_t T = qo[batch], n_idx = kvp[batch];
+  if (T * H > std::numeric_limits<int32_t>::max() - kTileM) return MLA_ERR_INVALID_ARGUMENT;
+  if (n_idx > kMaxPageIds) return MLA_ERR_INVALID_ARGUMENT;  // beyond the fixed scratch
+  if (n_idx > 0 && !kvi) return MLA_ERR_INVALID_ARGUMENT;
+  for (int64_t i = 0; i < n_idx; ++i)
+    if (kvi[i] < 0 || kvi[i] >= d.num_pages) return MLA_ERR_INVALID_ARGUMENT;
+  // pass 1: validate rows, count tiles
+  int64_t total_tiles = 0, n_tiles = 0;
+  const int32_t tok_per_tile = kTileM / H;
+  for (int32_t b = 0; b < batch; ++b) {
+    const int64_t n = kvp[b + 1] - kvp[b];
+    if (n > 0 ? (last[b] < 1 || last[b] > P) : (last[b] < 0 || last[b] > P)) return MLA_ERR_INVALID_ARGUMENT;
+    const int64_t k = n > 0 ? (n - 1) * P + last[b] : 0;
+    if (k > std::numeric_limits<int32_t>::max() - kTileN) return MLA_ERR_INVALID_ARGUMENT;
+    const int32_t q_b = qo[b + 1] - qo[b];
+    for (int32_t tok0 = 0; tok0 < q_b; tok0 += tok_per_tile) {
+      const int32_t ntok = std::min(tok_per_tile, q_b - tok0);
+      const int64_t diag = causal ? k - q_b + tok0 : k;
+      const int64_t hi = std::max<int64_t>(0, std::min<int64_t>(causal ? diag + ntok : k, k));
+      total_tiles += (hi + kTileN - 1) / kTileN;
+      ++n_tiles;
+    }
+  }
+  if (n_tiles > kMaxWork) return MLA_ERR_INVALID_ARGUMENT;  // beyond the fixed scratch
+  const int units = std::max(1, num_sms / 2);
+  const int64_t chunk = std::max<int64_t>(8, (total_tiles + units - 1) / units);
+  // pass 2: emit (every tile still to come keeps at least one work slot)
+  int nw = 0, nm = 0, np = 0;
+  int64_t tiles_left = n_tiles;
+  for (int32_t b = 0; b < batch; ++b) {
+    const int64_t n = kvp[b + 1] - kvp[b];
+    const int32_t k = n > 0 ? static_cast<int32_t>((n - 1) * P + last[b]) : 0;
+    const int32_t q_b = qo[b + 1] - qo[b];
+    for (int32_t tok0 = 0; tok0 < q_b; tok0 += tok_per_tile) {
+      const int32_t ntok = std::min(tok_per_tile, q_b - tok0);
+      const int32_t diag = causal ? k - q_b + tok0 : k;
+      const int64_t hi64 = std::max<int64_t>(0, std::min<int64_t>(causal ? int64_t(diag) + ntok : k, k));
+      const int32_t vis_hi = static_cast<int32_t>(hi64);
+      const int32_t nt = (vis_hi + kTileN - 1) / kTileN;
+      const int32_t q_row0 = (qo[b] + tok0) * H;
+      int32_t pieces = nt > chunk ? static_cast<int32_t>((nt + chunk - 1) / chunk) : 1;
+      --tiles_left;
+      if (pieces > 1 && (np + pieces > kMaxPartials || nm >= kMaxMerge ||
+                         nw + pieces + tiles_left > kMaxWork))
+        pieces = 1;  // no scratch left for partials: run this tile unsplit
+      if (nw + pieces > kMaxWork) return MLA_ERR_INVALID_ARGUMENT;
+      if (pieces == 1) {
+        g_work[nw++] = WorkItem{q_row0, ntok * H, kvp[b], k, 0, vis_hi, diag, -1};
+        continue;
+      }
+      g_merge[nm++] = MergeItem{q_row0, ntok * H, np, pieces};
+      for (int32_t i = 0; i < pieces; ++i) {
+        const int32_t lo = int32_t(int64_t(nt) * i / pieces), hi = int32_t(int64_t(nt) * (i + 1) / pieces);
+        g_work[nw++] = WorkItem{q_row0, ntok * H, kvp[b], k, lo * kTileN, std::min(hi * kTileN, vis_hi), diag, np + i};
+      }
+      np += pieces;
+    }
+  }
+  std::sort(g_work, g_work + nw, [](const WorkItem& a, const WorkItem& c) {
+    return (a.key_end - a.key_begin) > (c.key_end - c.key_begin);
+  });
+  *n_work = nw;
+  *n_merge = nm;
+  *n_partials = np;
+  *total_tokens = static_cast<int32_t>(T);
+  return MLA_OK;
+}
+
+}  // namespace
+
+// The scratch array itself.  Device code could name it directly; host code only ever
+// uses the address returned by cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_mla_noalloc_scratch[kScratchBytes];
+
+extern "C" mla_status mla_run_noalloc(const mla_dims* dims, int32_t batch, const int32_t* qo_indptr,
+                                      const int32_t* kv_indptr, const int32_t* kv_indices,
+                                      const int32_t* last_page_len, int32_t causal, const void* q_nope,
+                                      const void* q_pe, const void* cache, void* out, float* lse, void* stream) {
+  if (!dims || (causal != 0 && causal != 1)) return MLA_ERR_INVALID_ARGUMENT;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+
+  // One-time set-up on this device (with it current): the scratch array's device
+  // address, the SM count, and the driver's tensor-map encoder.
+  static EncodeTiledFn enc = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!g_dev[dev].ptr) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_mla_noalloc_scratch) != cudaSuccess || !ptr) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+      }
+      int sms = 0;
+      if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MLA_ERR_CUDA;
+      g_dev[dev].ptr = static_cast<unsigned char*>(ptr);
+      g_dev[dev].num_sms = sms;
+    }
+    if (!enc) {
+      void* f = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess)
+        return MLA_ERR_CUDA;
+      enc = reinterpret_cast<EncodeTiledFn>(f);
+    }
+  }
+  unsigned char* scratch = g_dev[dev].ptr;
+
+  int n_work = 0, n_merge = 0, n_partials = 0;
+  int32_t T = 0;
+  mla_status st = plan_fixed(*dims, batch, qo_indptr, kv_indptr, kv_indices, last_page_len, causal != 0,
+                             g_dev[dev].num_sms, &n_work, &n_merge, &n_partials, &T);
+  if (st != MLA_OK) return st;
+  if (n_work == 0) return MLA_OK;
+  if (!q_nope || !q_pe || !cache || !out) return MLA_ERR_INVALID_ARGUMENT;
+  auto misaligned = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) != 0; };
+  if (misaligned(q_nope) || misaligned(q_pe) || misaligned(cache) || misaligned(out) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return MLA_ERR_INVALID_ARGUMENT;
+
+  // Fill the scratch: status word cleared, work and merge lists, page-table copy.  The
+  // copies read host memory that is pageable, so each returns once its source has been
+  // read and the static host buffers may be reused by the next call.
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t n_idx = static_cast<size_t>(kv_indptr[batch]);
+  if (cudaMemsetAsync(scratch + kOffStatus, 0, 256, s) != cudaSuccess ||
+      cudaMemcpyAsync(scratch + kOffWork, g_work, sizeof(WorkItem) * n_work, cudaMemcpyHostToDevice, s) !=
+          cudaSuccess ||
+      (n_merge > 0 && cudaMemcpyAsync(scratch + kOffMerge, g_merge, sizeof(MergeItem) * n_merge,
+                                      cudaMemcpyHostToDevice, s) != cudaSuccess) ||
+      (n_idx > 0 && cudaMemcpyAsync(scratch + kOffPages, kv_indices, sizeof(int32_t) * n_idx,
+                                    cudaMemcpyHostToDevice, s) != cudaSuccess)) {
+    cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+
+  const int P = dims->page_size;
+  const uint64_t rows = uint64_t(T) * dims->num_heads;
+  const uint64_t cache_rows = uint64_t(dims->num_pages) * P;
+  const uint32_t box_rows = P < kTileN ? P : kTileN;
+  CUtensorMap tm_q, tm_qpe, tm_kv, tm_kpe;
+  if (!encode_2d(enc, &tm_q, q_nope, rows, kCkv, 64, kTileM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(enc, &tm_qpe, q_pe, rows, kRope, 32, kTileM, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !encode_2d(enc, &tm_kv, cache, cache_rows, kLatent, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(enc, &tm_kpe, cache, cache_rows, kLatent, 32, box_rows, CU_TENSOR_MAP_SWIZZLE_64B))
+    return MLA_ERR_CUDA;
+
+  float* partials = reinterpret_cast<float*>(scratch + kOffPartials);
+  AttnParams ap;
+  ap.work = reinterpret_cast<const WorkItem*>(scratch + kOffWork);
+  ap.kv_indices = reinterpret_cast<const int32_t*>(scratch + kOffPages);
+  ap.q_nope = q_nope;
+  ap.q_pe = q_pe;
+  ap.total_rows = static_cast<int32_t>(rows);
+  ap.out = out;
+  ap.lse = lse;
+  ap.ws_o = partials;
+  ap.ws_lse = partials + size_t(n_partials) * kTileM * kCkv;
+  ap.status = reinterpret_cast<int32_t*>(scratch + kOffStatus);
+  ap.scale_log2 = dims->sm_scale * 1.4426950408889634f;
+  ap.num_heads = dims->num_heads;
+  ap.page_size = P;
+  ap.box_rows = static_cast<int32_t>(box_rows);
+  ap.timeout_ns = 4000000000ull;
+  ap.debug_flags = 0;
+  if (launch_attention(tm_q, tm_qpe, tm_kv, tm_kpe, ap, n_work, s) != cudaSuccess) return MLA_ERR_CUDA;
+  if (n_merge > 0) {
+    MergeParams mp{reinterpret_cast<const MergeItem*>(scratch + kOffMerge), ap.ws_o, ap.ws_lse, out, lse};
+    if (launch_merge(mp, n_merge, s) != cudaSuccess) return MLA_ERR_CUDA;
+  }
+  return MLA_OK;
+}
