@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <limits>
 #include <mutex>
 #include <new>
 
@@ -224,6 +225,7 @@ mla_status mla_run(mla_plan_t p, const void* q_nope, const void* q_pe, const voi
   ap.ws_lse = p->d_ws ? p->d_ws + static_cast<size_t>(p->layout.num_partials) * kTileM * kCkv : nullptr;
   ap.status = p->d_status;
   ap.scale_log2 = p->dims.sm_scale * 1.4426950408889634f;
+  ap.nan_guard = std::numeric_limits<float>::quiet_NaN();
   ap.num_heads = p->dims.num_heads;
   ap.page_size = P;
   ap.box_rows = static_cast<int32_t>(box_rows);

@@ -434,10 +434,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         t[4 * c + 2] = __uint_as_float(sr[4 * c + 2]) + x.z;
         t[4 * c + 3] = __uint_as_float(sr[4 * c + 3]) + x.w;
       }
-      // Every lane has consumed its loaded values (the sums above), so the slot can be
-      // handed back with a relaxed arrive.
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote_relaxed(bar(bXEmpty + 4 * xsl + q), peer);
 
       // --- mask (partial tiles only), running max in the log2 domain, lazy rescale
       const int nvalid = lim - (w.key_begin + kTileN * j);
@@ -455,6 +451,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float mt = mraw * scale;  // scale > 0 keeps the order; -inf stays -inf
+      // Hand the slot back to the peer.  mraw depends on every value loaded from the
+      // slot, and the vote needs every lane's mraw, so all of this warp's loads have
+      // delivered their data before lane 0's arrive issues; the peer's next push cannot
+      // overtake them.  (An arrive issued before the loads completed did let it; a
+      // release-ordered arrive also works but costs a cluster-scope fence per tile.)
+      if (__any_sync(0xffffffffu, mraw != p.nan_guard) && lane == 0)
+        mbar_arrive_remote_relaxed(bar(bXEmpty + 4 * xsl + q), peer);
       // Keep the old reference max unless the new one exceeds it by more than 8 (a
       // factor of 256 in the weights); then rescale the running sum and output row.
       const bool bump = mt > m_run + 8.f;

@@ -22,6 +22,8 @@ struct AttnParams {
   float* ws_lse;   // fp32 [partials, 128]
   int32_t* status; // device status word
   float scale_log2;  // sm_scale * log2(e)
+  float nan_guard;   // always NaN: `x != nan_guard` is true for every x, yet the compiler
+                     // cannot fold it, so a vote on it waits for x to be computed
   int32_t num_heads;
   int32_t page_size;
   int32_t box_rows;  // min(page_size, 64)

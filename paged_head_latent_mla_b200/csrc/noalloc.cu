@@ -250,6 +250,7 @@ extern "C" mla_status mla_run_noalloc(const mla_dims* dims, int32_t batch, const
   ap.ws_lse = partials + size_t(n_partials) * kTileM * kCkv;
   ap.status = reinterpret_cast<int32_t*>(scratch + kOffStatus);
   ap.scale_log2 = dims->sm_scale * 1.4426950408889634f;
+  ap.nan_guard = std::numeric_limits<float>::quiet_NaN();
   ap.num_heads = dims->num_heads;
   ap.page_size = P;
   ap.box_rows = static_cast<int32_t>(box_rows);
