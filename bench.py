@@ -391,6 +391,22 @@ def summarise(d, res, peaks):
     }
 
 
+def reduce_max_over_ranks(x: float, dist, device) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    if dist is None:
+        return x
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job GB/s: every rank's bytes over the slowest rank's time."""
+    return world * bytes_per_rank / (ms_max * 1e-3) / 1e9
+
+
 def run_native(args):
     import torch
 
@@ -421,22 +437,15 @@ def run_native(args):
     sampler = ClockSampler(local)
     res = time_workload(d, device, args.steps, max(3, args.warmup), dist=dist, soak_s=args.soak, sampler=sampler,
                         copies=args.copies)
-    ms = res["ms_per_step"]
-    if dist is not None:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * w["kv_bytes"] / (ms * 1e-3) / 1e9
+    ms = reduce_max_over_ranks(res["ms_per_step"], dist, device)
+    value = job_throughput(w["kv_bytes"], world, ms)
     summ = summarise(d, res, peaks)
 
     e2e = None
     if not args.no_e2e:
         e2e_ms, h2d, d2h = time_e2e(d, device, max(5, min(args.steps, 30)), 3)
-        if dist is not None:
-            t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * w["kv_bytes"] / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e2e_ms = reduce_max_over_ranks(e2e_ms, dist, device)
+        e2e = {"value": job_throughput(w["kv_bytes"], world, e2e_ms), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms,
                "includes": "mla_plan from host tables + H2D of queries + mla_run + D2H of out/lse + status read"}
 
