@@ -63,18 +63,21 @@ typedef struct {
 /* Optional planning knobs; pass NULL for the defaults (all zero). */
 typedef struct {
   int32_t split_keys;       /* 0: automatic split-KV; > 0: cut every key range into
-                               chunks of this many keys (a multiple of 64); < 0: never
-                               split                                                  */
+                               chunks of this many keys (a multiple of MLA_KEY_TILE);
+                               < 0: never split                                       */
   int32_t num_sms;          /* 0: query the device; > 0: plan for this many SMs       */
   uint64_t wait_timeout_ns; /* bound on every in-kernel wait; 0: 4 seconds            */
   int32_t debug_flags;      /* bit 0 (MLA_DEBUG_DROP_FIRST_KV_LOAD): the kernel never
-                               loads its first key tile, so the wait on it runs out and
+                               loads its first key chunk, so the wait on it runs out and
                                the run reports MLA_ERR_DEVICE_TIMEOUT (tests the
                                timeout path without faulting anything)                */
   int32_t host_only;        /* 1: build the work lists on the host only, touching no
                                CUDA API (for inspecting a plan on a machine without a
                                GPU); such a plan can be described but not run         */
 } mla_plan_options;
+
+/* Keys per tile of the attention kernel: work items start on multiples of it. */
+#define MLA_KEY_TILE 64
 
 #define MLA_DEBUG_DROP_FIRST_KV_LOAD 1
 #define MLA_DEBUG_KERNEL_TIMING 2 /* bit 1: mla_run records CUDA events around each of its

@@ -28,6 +28,7 @@ MLA_ERR_UNSUPPORTED = 2
 MLA_ERR_CUDA = 3
 MLA_ERR_OUT_OF_MEMORY = 4
 MLA_ERR_DEVICE_TIMEOUT = 5
+MLA_KEY_TILE = 64  # keys per kernel tile; split sizes are multiples of it
 MLA_DEBUG_DROP_FIRST_KV_LOAD = 1
 MLA_DEBUG_KERNEL_TIMING = 2
 WORK_FIELDS = 8

@@ -1,5 +1,5 @@
-// C ABI of the paged latent-attention library: plan ownership, tensor-map encoding,
-// launches and the device status word.  See include/mla.h for the contract.
+// C ABI of the paged latent-attention library: plan ownership, launches and the device
+// status word.  See include/mla.h for the contract.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -31,7 +31,7 @@ struct mla_plan_s {
   WorkItem* d_work = nullptr;
   MergeItem* d_merge = nullptr;
   int32_t* d_kv_indices = nullptr;
-  float* d_ws = nullptr;  // [partials * 128 * 512] o, then [partials * 128] lse
+  uint8_t* d_ws = nullptr;  // [partials][128][512] bf16 o, then [partials][128] fp32 lse
   void* h_staging = nullptr;
   cudaEvent_t ev_last = nullptr;
   // kernel timing ring (MLA_DEBUG_KERNEL_TIMING): 3 events per run
@@ -41,38 +41,6 @@ struct mla_plan_s {
 };
 
 namespace {
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static std::once_flag once;
-  static EncodeTiledFn fn = nullptr;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(f);
-  });
-  return fn;
-}
-
-// 2-D bf16 tensor map over a row-major [rows, cols] matrix with row pitch `pitch_elems`.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_elems,
-              uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {pitch_elems * 2};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t es[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -169,8 +137,8 @@ mla_status mla_plan(const mla_dims* dims, int32_t batch, const int32_t* qo_indpt
   p->d_merge = reinterpret_cast<MergeItem*>(d + off_merge);
   p->d_kv_indices = reinterpret_cast<int32_t*>(d + off_idx);
   if (p->layout.num_partials > 0) {
-    const size_t ws = static_cast<size_t>(p->layout.num_partials) * kTileM * (kCkv + 1) * sizeof(float);
-    if (cudaMalloc(&p->d_ws, ws) != cudaSuccess) { cudaGetLastError(); free_plan(p); return MLA_ERR_OUT_OF_MEMORY; }
+    const size_t ws = static_cast<size_t>(p->layout.num_partials) * kPartialBytes;
+    if (cudaMalloc(reinterpret_cast<void**>(&p->d_ws), ws) != cudaSuccess) { cudaGetLastError(); free_plan(p); return MLA_ERR_OUT_OF_MEMORY; }
   }
   if (p->opts.debug_flags & MLA_DEBUG_KERNEL_TIMING) {
     p->ring = new (std::nothrow) cudaEvent_t[3 * mla_plan_s::kRing]();
@@ -203,37 +171,30 @@ mla_status mla_run(mla_plan_t p, const void* q_nope, const void* q_pe, const voi
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev != p->device) return MLA_ERR_INVALID_ARGUMENT;
 
-  const int P = p->dims.page_size;
-  CUtensorMap tm_q, tm_qpe, tm_kv, tm_kpe;
-  const uint64_t cache_rows = static_cast<uint64_t>(p->dims.num_pages) * P;
-  const uint32_t box_rows = P < kTileN ? P : kTileN;
-  if (!make_map(&tm_q, q_nope, rows, kCkv, kCkv, 64, kTileM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&tm_qpe, q_pe, rows, kRope, kRope, 32, kTileM, CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_map(&tm_kv, cache, cache_rows, kLatent, kLatent, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&tm_kpe, cache, cache_rows, kLatent, kLatent, 32, box_rows, CU_TENSOR_MAP_SWIZZLE_64B))
-    return MLA_ERR_CUDA;
-
-  AttnParams ap;
+  AttnLaunch a;
+  AttnParams& ap = a.p;
   ap.work = p->d_work;
   ap.kv_indices = p->d_kv_indices;
-  ap.q_nope = q_nope;
-  ap.q_pe = q_pe;
-  ap.total_rows = static_cast<int32_t>(rows);
   ap.out = out;
   ap.lse = lse;
   ap.ws_o = p->d_ws;
-  ap.ws_lse = p->d_ws ? p->d_ws + static_cast<size_t>(p->layout.num_partials) * kTileM * kCkv : nullptr;
+  ap.ws_lse = p->d_ws ? reinterpret_cast<float*>(p->d_ws + static_cast<size_t>(p->layout.num_partials) * kPartialOBytes)
+                      : nullptr;
   ap.status = p->d_status;
   ap.scale_log2 = p->dims.sm_scale * 1.4426950408889634f;
-  ap.nan_guard = std::numeric_limits<float>::quiet_NaN();
   ap.num_heads = p->dims.num_heads;
-  ap.page_size = P;
-  ap.box_rows = static_cast<int32_t>(box_rows);
+  ap.page_size = p->dims.page_size;
   ap.timeout_ns = p->opts.wait_timeout_ns ? p->opts.wait_timeout_ns : 4000000000ull;
   ap.debug_flags = p->opts.debug_flags;
+  a.q_nope = q_nope;
+  a.q_pe = q_pe;
+  a.cache = cache;
+  a.rows = static_cast<uint64_t>(rows);
+  a.cache_rows = static_cast<uint64_t>(p->dims.num_pages) * p->dims.page_size;
+  a.num_work = static_cast<int>(p->layout.work.size());
   cudaEvent_t* ev = p->ring ? p->ring + 3 * (p->runs % mla_plan_s::kRing) : nullptr;
   if (ev && cudaEventRecord(ev[0], s) != cudaSuccess) return MLA_ERR_CUDA;
-  cudaError_t e = launch_attention(tm_q, tm_qpe, tm_kv, tm_kpe, ap, static_cast<int>(p->layout.work.size()), s);
+  cudaError_t e = launch_attention(a, s);
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   if (ev && cudaEventRecord(ev[1], s) != cudaSuccess) return MLA_ERR_CUDA;
   if (!p->layout.merge.empty()) {
@@ -273,7 +234,7 @@ mla_status mla_plan_get_info(mla_plan_t p, mla_plan_info* info) {
   info->num_merge = static_cast<int32_t>(p->layout.merge.size());
   info->num_partials = p->layout.num_partials;
   info->num_sms = p->opts.num_sms;
-  info->workspace_bytes = static_cast<int64_t>(p->layout.num_partials) * kTileM * (kCkv + 1) * 4;
+  info->workspace_bytes = static_cast<int64_t>(p->layout.num_partials) * static_cast<int64_t>(kPartialBytes);
   return MLA_OK;
 }
 

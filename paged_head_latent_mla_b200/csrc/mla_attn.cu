@@ -33,6 +33,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "mla_internal.h"
 #include "mla_launch.h"
@@ -141,6 +142,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   const uint32_t sb = smem_addr(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank(), peer = rank ^ 1u;
+  // A merge grid launched after this one may be scheduled as SMs free up; it waits for
+  // this grid to finish before reading anything.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const WorkItem w = p.work[blockIdx.x >> 1];
   const int ntiles = w.key_end > w.key_begin ? (w.key_end - w.key_begin + kTileN - 1) / kTileN : 0;
 
@@ -507,61 +511,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       if (lane == 0) mbar_arrive(bar(bPFull + b2));
     }
 
-    // --- epilogue
+    // --- epilogue.  Each warp stages its 32 rows of O / l (bf16) in the KV ring (idle now:
+    // every load was consumed by a finished PV) and writes them back one 512-byte half
+    // row per warp store, so every store covers whole cache lines.  16-byte piece c of staged row R sits at
+    // position c ^ R, which keeps both the row-wise writes and the piece-wise reads free
+    // of bank conflicts.
     if (ok) {
       const bool has = l_run > 0.f;
       const float inv_l = has ? 1.f / l_run : 0.f;
       const float lse_nat = has ? (m_run + __log2f(l_run)) * 0.69314718055994531f : kNegInf;
-      const bool row_ok = r < w.n_rows;
       if (ntiles > 0) {
         ok = wait_warp(bar(bPVDone + ((ntiles - 1) & 1)), ((ntiles - 1) >> 1) & 1, kSiteEpilogue, false);
         tc_fence_after();
       }
       if (ok) {
-        if (w.partial < 0) {
-          __nv_bfloat16* dst =
-              static_cast<__nv_bfloat16*>(p.out) + static_cast<size_t>(w.q_row0 + r) * kCkv + 256 * rank;
-          for (int cc = 0; cc < 256; cc += 32) {
-            uint32_t o[32];
-            if (ntiles > 0) {
-              tmem_ld32(trow + kColO + cc, o);
-              tmem_wait_ld();
-            } else {
+        const bool part = w.partial >= 0;  // bf16 partial in the workspace, or the output
+        uint8_t* stage = smem + kKV + q * 16384;  // 32 rows x 512 B
+        for (int cc = 0; cc < 256; cc += 32) {
+          uint32_t o[32];
+          if (ntiles > 0) {
+            tmem_ld32(trow + kColO + cc, o);
+          } else {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = 0u;
-            }
-            if (row_ok) {
-              uint4 v[4];
-              uint32_t* vp = reinterpret_cast<uint32_t*>(v);
-#pragma unroll
-              for (int i = 0; i < 16; ++i)
-                vp[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-              uint4* d4 = reinterpret_cast<uint4*>(dst + cc);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) d4[i] = v[i];
-            }
+            for (int i = 0; i < 32; ++i) o[i] = 0u;
           }
-          if (rank == 0 && p.lse != nullptr && row_ok) p.lse[w.q_row0 + r] = lse_nat;
-        } else {
-          float* dst = p.ws_o + (static_cast<size_t>(w.partial) * kTileM + r) * kCkv + 256 * rank;
-          for (int cc = 0; cc < 256; cc += 32) {
-            uint32_t o[32];
-            if (ntiles > 0) {
-              tmem_ld32(trow + kColO + cc, o);
-              tmem_wait_ld();
-            } else {
+          uint8_t* row = stage + (lane << 9);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = 0u;
-            }
-            if (row_ok) {
-              float4* d4 = reinterpret_cast<float4*>(dst + cc);
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                d4[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l, __uint_as_float(o[4 * i + 1]) * inv_l,
-                                    __uint_as_float(o[4 * i + 2]) * inv_l, __uint_as_float(o[4 * i + 3]) * inv_l);
-            }
+          for (int i = 0; i < 4; ++i) {
+            const int c = (cc >> 3) + i;  // pieces of 8 bf16
+            *reinterpret_cast<uint4*>(row + ((c ^ lane) << 4)) = make_uint4(
+                pack_bf16x2(__uint_as_float(o[8 * i + 0]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l),
+                pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l),
+                pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l),
+                pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l));
           }
-          if (rank == 0 && row_ok) p.ws_lse[static_cast<size_t>(w.partial) * kTileM + r] = lse_nat;
+        }
+        __syncwarp();
+        const int nrows = min(32, w.n_rows - 32 * q);  // rows of this warp inside the tile
+        uint8_t* base = part ? static_cast<uint8_t*>(p.ws_o) + static_cast<size_t>(w.partial) * kTileM * kCkv * 2
+                             : static_cast<uint8_t*>(p.out) + static_cast<size_t>(w.q_row0) * kCkv * 2;
+        for (int R = 0; R < nrows; ++R) {
+          uint8_t* dst = base + (static_cast<size_t>(32 * q + R) * kCkv + 256 * rank) * 2;
+          *reinterpret_cast<uint4*>(dst + (lane << 4)) =
+              *reinterpret_cast<const uint4*>(stage + (R << 9) + ((lane ^ R) << 4));
+        }
+        if (rank == 0 && r < w.n_rows) {
+          if (!part) {
+            if (p.lse != nullptr) p.lse[w.q_row0 + r] = lse_nat;
+          } else {
+            p.ws_lse[static_cast<size_t>(w.partial) * kTileM + r] = lse_nat;
+          }
         }
       }
     }
@@ -579,55 +578,116 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   cluster_wait();
 }
 
-// Combine the fp32 partials of split query tiles by their log-sum-exp:
+// Combine the partials of split query tiles by their log-sum-exp:
 // M = max_i lse_i, out = sum_i e^{lse_i - M} o_i / sum_i e^{lse_i - M},
 // lse = M + ln sum_i e^{lse_i - M} (FlashInferMLAManager.run: merging key segments).
+// One warp per row; lane l owns columns [16l, 16l + 16), so every load and store of a
+// row is one contiguous 1 KB access; four partials are in flight at a time.
 __global__ void __launch_bounds__(256) mla_merge_kernel(const MergeParams p) {
-  // 16 blocks per split query tile, 8 rows (one per warp) per block.
-  const MergeItem m = p.merge[blockIdx.x >> 4];
+  // Launched as a programmatic dependent of the attention grid: wait until that grid has
+  // finished and its partials are visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const MergeItem m = p.merge[blockIdx.x >> 4];  // 16 blocks per split query tile
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = ((blockIdx.x & 15) << 3) + warp;
-  if (r < m.n_rows) {
-    float M = -__int_as_float(0x7f800000);
-    for (int i = 0; i < m.n_partials; ++i)
-      M = fmaxf(M, p.ws_lse[static_cast<size_t>(m.first_partial + i) * kTileM + r]);
-    float4 acc[4];
+  const int r = ((blockIdx.x & 15) << 3) + warp;  // 8 rows (one per warp) per block
+  if (r >= m.n_rows) return;
+  const float neg_inf = -__int_as_float(0x7f800000);
+  const int n = m.n_partials;
+  float M = neg_inf;
+  for (int i = lane; i < n; i += 32) M = fmaxf(M, p.ws_lse[static_cast<size_t>(m.first_partial + i) * kTileM + r]);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-    float z = 0.f;
-    if (M != -__int_as_float(0x7f800000)) {
-      for (int i = 0; i < m.n_partials; ++i) {
-        const size_t slot = static_cast<size_t>(m.first_partial + i) * kTileM + r;
-        const float wgt = __expf(p.ws_lse[slot] - M);
-        z += wgt;
-        const float4* src = reinterpret_cast<const float4*>(p.ws_o + slot * kCkv);
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  float acc[16];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float4 v = src[lane + 32 * k];
-          acc[k].x += wgt * v.x;
-          acc[k].y += wgt * v.y;
-          acc[k].z += wgt * v.z;
-          acc[k].w += wgt * v.w;
+  for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+  float z = 0.f;
+  if (M != neg_inf) {
+    for (int i0 = 0; i0 < n; i0 += 32) {
+      const int cnt = min(32, n - i0);
+      // lane u holds the weight of partial i0 + u
+      const float wl =
+          lane < cnt ? __expf(p.ws_lse[static_cast<size_t>(m.first_partial + i0 + lane) * kTileM + r] - M) : 0.f;
+      z += wl;
+      for (int k = 0; k < cnt; k += 4) {
+        uint4 v[4][2];
+        float wk[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          wk[u] = __shfl_sync(0xffffffffu, wl, k + u);  // k + u <= 31
+          if (k + u < cnt) {
+            const uint4* src = reinterpret_cast<const uint4*>(
+                static_cast<const uint8_t*>(p.ws_o) +
+                ((static_cast<size_t>(m.first_partial + i0 + k + u) * kTileM + r) * kCkv + 16 * lane) * 2);
+            v[u][0] = src[0];
+            v[u][1] = src[1];
+          } else {
+            v[u][0] = v[u][1] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t* wv = reinterpret_cast<const uint32_t*>(v[u]);
+#pragma unroll
+          for (int k2 = 0; k2 < 8; ++k2) {
+            acc[2 * k2] += wk[u] * __uint_as_float(wv[k2] << 16);
+            acc[2 * k2 + 1] += wk[u] * __uint_as_float(wv[k2] & 0xffff0000u);
+          }
         }
       }
     }
-    const float inv = z > 0.f ? 1.f / z : 0.f;
-    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + static_cast<size_t>(m.q_row0 + r) * kCkv;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      uint2 v;
-      v.x = ptx::pack_bf16x2(acc[k].x * inv, acc[k].y * inv);
-      v.y = ptx::pack_bf16x2(acc[k].z * inv, acc[k].w * inv);
-      *reinterpret_cast<uint2*>(dst + 4 * (lane + 32 * k)) = v;
-    }
-    if (p.lse != nullptr && lane == 0)
-      p.lse[m.q_row0 + r] = z > 0.f ? M + __logf(z) : -__int_as_float(0x7f800000);
+    for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
   }
+  const float inv = z > 0.f ? 1.f / z : 0.f;
+  uint4 o[2];
+  uint32_t* ov = reinterpret_cast<uint32_t*>(o);
+#pragma unroll
+  for (int k2 = 0; k2 < 8; ++k2) ov[k2] = ptx::pack_bf16x2(acc[2 * k2] * inv, acc[2 * k2 + 1] * inv);
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + static_cast<size_t>(m.q_row0 + r) * kCkv +
+                                        16 * lane);
+  dst[0] = o[0];
+  dst[1] = o[1];
+  if (p.lse != nullptr && lane == 0) p.lse[m.q_row0 + r] = z > 0.f ? M + __logf(z) : neg_inf;
 }
 
 // ---------------------------------------------------------------------- launchers
-cudaError_t launch_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_qpe, const CUtensorMap& tm_kv,
-                             const CUtensorMap& tm_kpe, const AttnParams& p, int num_work, cudaStream_t stream) {
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix (row pitch = cols).
+bool encode_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+               uint32_t box_rows, CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
   static thread_local int configured_device = -1;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -638,13 +698,36 @@ cudaError_t launch_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_qpe,
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  mla_attn_kernel<<<2 * num_work, attn::kThreads, attn::kSmemAlloc, stream>>>(tm_q, tm_qpe, tm_kv, tm_kpe, p);
+  AttnParams p = a.p;
+  p.q_nope = a.q_nope;
+  p.q_pe = a.q_pe;
+  p.nan_guard = __builtin_nanf("");
+  p.box_rows = p.page_size < kTileN ? p.page_size : kTileN;
+  const uint32_t br = static_cast<uint32_t>(p.box_rows);
+  CUtensorMap tm_q, tm_qpe, tm_kv, tm_kpe;
+  if (!encode_2d(&tm_q, a.q_nope, a.rows, kCkv, 64, kTileM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&tm_qpe, a.q_pe, a.rows, kRope, 32, kTileM, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !encode_2d(&tm_kv, a.cache, a.cache_rows, kLatent, 64, br, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&tm_kpe, a.cache, a.cache_rows, kLatent, 32, br, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  mla_attn_kernel<<<2 * a.num_work, attn::kThreads, attn::kSmemAlloc, stream>>>(tm_q, tm_qpe, tm_kv, tm_kpe, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_merge(const MergeParams& p, int num_merge, cudaStream_t stream) {
-  mla_merge_kernel<<<num_merge * 16, 256, 0, stream>>>(p);
-  return cudaGetLastError();
+  // Programmatic dependent launch: the merge grid is set up while the attention grid
+  // drains, and its griddepcontrol.wait releases it once that grid has finished.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(num_merge) * 16u);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mla_merge_kernel, p);
 }
 
 }  // namespace mla

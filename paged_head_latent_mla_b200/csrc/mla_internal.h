@@ -12,7 +12,11 @@ constexpr int kLatent = 576;   // ckv 512 | kpe 64
 constexpr int kCkv = 512;
 constexpr int kRope = 64;
 constexpr int kTileM = 128;    // query rows per tile (tokens x heads)
-constexpr int kTileN = 64;     // keys per tile
+constexpr int kTileN = MLA_KEY_TILE;  // keys per tile (64)
+// Split-KV workspace per partial: the 128 x 512 output tile in bf16, then its 128 fp32
+// log-sum-exps (all partials' tiles first, then all their lse rows).
+constexpr size_t kPartialOBytes = size_t(kTileM) * kCkv * 2;
+constexpr size_t kPartialBytes = kPartialOBytes + size_t(kTileM) * 4;
 
 // One unit of attention work: a 128-row query tile against keys [key_begin, key_end)
 // of one batch row.  Processed by one CTA pair; field order matches mla_plan_describe.
@@ -21,7 +25,7 @@ struct WorkItem {
   int32_t n_rows;     // valid rows in the tile (tokens_in_tile * H)
   int32_t page_base;  // kv_indptr[b]: the row's first entry in kv_indices
   int32_t kv_len;     // k_b
-  int32_t key_begin;  // multiple of 64
+  int32_t key_begin;  // multiple of kTileN
   int32_t key_end;    // exclusive
   int32_t diag_base;  // row r sees keys < clamp(diag_base + r / H + 1, 0, kv_len)
   int32_t partial;    // -1: final output; else workspace slot

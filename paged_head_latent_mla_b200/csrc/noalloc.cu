@@ -40,7 +40,6 @@ constexpr size_t kOffWork = 256;
 constexpr size_t kOffMerge = kOffWork + sizeof(WorkItem) * kMaxWork;
 constexpr size_t kOffPages = kOffMerge + sizeof(MergeItem) * kMaxMerge;
 constexpr size_t kOffPartials = (kOffPages + sizeof(int32_t) * kMaxPageIds + 255) / 256 * 256;
-constexpr size_t kPartialBytes = size_t(kTileM) * (kCkv + 1) * sizeof(float);  // o + lse of one tile
 constexpr int kMaxPartials = static_cast<int>((kScratchBytes - kOffPartials) / kPartialBytes);
 static_assert(kMaxPartials >= 32, "scratch too small for useful splitting");
 
@@ -56,21 +55,6 @@ struct DeviceScratch {
 constexpr int kMaxDevices = 64;
 DeviceScratch g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-bool encode_2d(EncodeTiledFn enc, CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-               uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t es[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 // Validate the tables and cut the work into g_work / g_merge without allocating.
 // Long key ranges are split into chunks of about (total tiles / SM pairs) tiles while
@@ -171,8 +155,7 @@ extern "C" mla_status mla_run_noalloc(const mla_dims* dims, int32_t batch, const
   if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
 
   // One-time set-up on this device (with it current): the scratch array's device
-  // address, the SM count, and the driver's tensor-map encoder.
-  static EncodeTiledFn enc = nullptr;
+  // address and the SM count.
   {
     std::lock_guard<std::mutex> lock(g_dev_mutex);
     if (!g_dev[dev].ptr) {
@@ -185,15 +168,6 @@ extern "C" mla_status mla_run_noalloc(const mla_dims* dims, int32_t batch, const
       if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MLA_ERR_CUDA;
       g_dev[dev].ptr = static_cast<unsigned char*>(ptr);
       g_dev[dev].num_sms = sms;
-    }
-    if (!enc) {
-      void* f = nullptr;
-      cudaDriverEntryPointQueryResult q;
-      if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) !=
-              cudaSuccess ||
-          q != cudaDriverEntryPointSuccess)
-        return MLA_ERR_CUDA;
-      enc = reinterpret_cast<EncodeTiledFn>(f);
     }
   }
   unsigned char* scratch = g_dev[dev].ptr;
@@ -226,37 +200,28 @@ extern "C" mla_status mla_run_noalloc(const mla_dims* dims, int32_t batch, const
     return MLA_ERR_CUDA;
   }
 
-  const int P = dims->page_size;
-  const uint64_t rows = uint64_t(T) * dims->num_heads;
-  const uint64_t cache_rows = uint64_t(dims->num_pages) * P;
-  const uint32_t box_rows = P < kTileN ? P : kTileN;
-  CUtensorMap tm_q, tm_qpe, tm_kv, tm_kpe;
-  if (!encode_2d(enc, &tm_q, q_nope, rows, kCkv, 64, kTileM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_2d(enc, &tm_qpe, q_pe, rows, kRope, 32, kTileM, CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !encode_2d(enc, &tm_kv, cache, cache_rows, kLatent, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_2d(enc, &tm_kpe, cache, cache_rows, kLatent, 32, box_rows, CU_TENSOR_MAP_SWIZZLE_64B))
-    return MLA_ERR_CUDA;
-
-  float* partials = reinterpret_cast<float*>(scratch + kOffPartials);
-  AttnParams ap;
+  unsigned char* partials = scratch + kOffPartials;
+  AttnLaunch a;
+  AttnParams& ap = a.p;
   ap.work = reinterpret_cast<const WorkItem*>(scratch + kOffWork);
   ap.kv_indices = reinterpret_cast<const int32_t*>(scratch + kOffPages);
-  ap.q_nope = q_nope;
-  ap.q_pe = q_pe;
-  ap.total_rows = static_cast<int32_t>(rows);
   ap.out = out;
   ap.lse = lse;
   ap.ws_o = partials;
-  ap.ws_lse = partials + size_t(n_partials) * kTileM * kCkv;
+  ap.ws_lse = reinterpret_cast<float*>(partials + size_t(n_partials) * kPartialOBytes);
   ap.status = reinterpret_cast<int32_t*>(scratch + kOffStatus);
   ap.scale_log2 = dims->sm_scale * 1.4426950408889634f;
-  ap.nan_guard = std::numeric_limits<float>::quiet_NaN();
   ap.num_heads = dims->num_heads;
-  ap.page_size = P;
-  ap.box_rows = static_cast<int32_t>(box_rows);
+  ap.page_size = dims->page_size;
   ap.timeout_ns = 4000000000ull;
   ap.debug_flags = 0;
-  if (launch_attention(tm_q, tm_qpe, tm_kv, tm_kpe, ap, n_work, s) != cudaSuccess) return MLA_ERR_CUDA;
+  a.q_nope = q_nope;
+  a.q_pe = q_pe;
+  a.cache = cache;
+  a.rows = uint64_t(T) * dims->num_heads;
+  a.cache_rows = uint64_t(dims->num_pages) * dims->page_size;
+  a.num_work = n_work;
+  if (launch_attention(a, s) != cudaSuccess) return MLA_ERR_CUDA;
   if (n_merge > 0) {
     MergeParams mp{reinterpret_cast<const MergeItem*>(scratch + kOffMerge), ap.ws_o, ap.ws_lse, out, lse};
     if (launch_merge(mp, n_merge, s) != cudaSuccess) return MLA_ERR_CUDA;

@@ -30,9 +30,9 @@ struct QTile {
   int32_t q_row0, n_rows, page_base, kv_len, diag_base, vis_hi, ntiles;
 };
 
-// Cost, in units of one 64-key tile step, of the fixed work of one item: query
-// load, pipeline fill/drain and epilogue.  Split items also write an fp32 partial
-// that the merge kernel reads back.
+// Cost, in units of one key tile step, of the fixed work of one item: query load,
+// pipeline fill/drain and epilogue.  Split items also write an fp32 partial that the
+// merge kernel reads back.
 constexpr double kItemCost = 3.0;
 constexpr double kSplitCost = 2.0;
 

@@ -86,7 +86,7 @@ def test_host_plan_basic():
         dict(last_page_len=[0, 16]),  # row with pages needs >= 1
         dict(last_page_len=[5, 17]),
         dict(num_pages=0),
-        dict(split_keys=100),  # not a multiple of 64
+        dict(split_keys=100),  # not a multiple of the key tile
         dict(sm_scale=float("nan")),
     ],
 )

@@ -41,7 +41,7 @@ def check_layout(d, desc, num_sms=148):
         assert row_of_token[t0 + ntok - 1] == b, "a tile crosses batch rows"
         assert page_base == kvp[b]  # so key j -> kv_indices[page_base + j // P], slot j % P
         assert kv_len == k_oracle[b]
-        assert kb % 64 == 0 and kb <= ke or (kb == 0 and ke == 0)
+        assert kb % M.MLA_KEY_TILE == 0 and kb <= ke or (kb == 0 and ke == 0)
         q_b = qo[b + 1] - qo[b]
         i0 = t0 - qo[b]
         vis_hi = O.visible_keys(int(k_oracle[b]), int(q_b), int(i0 + ntok - 1), d.causal)
@@ -77,7 +77,7 @@ def check_layout(d, desc, num_sms=148):
         assert all(w[0] == q_row0 and w[1] == n_rows for w in items)
         spans = sorted((w[4], w[5]) for w in items)
         for a, b2 in zip(spans, spans[1:]):
-            assert a[1] == b2[0] and a[1] % 64 == 0
+            assert a[1] == b2[0] and a[1] % M.MLA_KEY_TILE == 0
     return True
 
 
@@ -135,7 +135,8 @@ def test_auto_split_balances_long_decode():
     assert desc["info"]["num_merge"] == 16  # every long row is split
     assert max(lens) <= 32768 // 4
     # balanced: total key tiles over 74 pairs vs the largest item
-    assert max(lens) / 64 <= 2 * (sum(lens) / 64) / 74 + 8
+    T = M.MLA_KEY_TILE
+    assert max(lens) / T <= 2 * (sum(lens) / T) / 74 + 8
 
 
 def test_no_split_for_small_decode():
