@@ -227,7 +227,9 @@ def run_reference(args):
 # ------------------------------------------------------------------------------- native leg
 def make_runner(d, device, n_copies, timing=True):
     """Plan once; keep `n_copies` copies of the inputs in HBM and rotate through them so
-    consecutive steps never find their inputs in L2."""
+    consecutive steps never find their inputs in L2.  With `timing` the plan records CUDA
+    events around each of its launches (kernel durations for the roofline); those events
+    sit between the attention and merge launches, so headline steps use a plan without."""
     import ctypes
 
     import torch
@@ -265,6 +267,9 @@ def input_bytes(d):
 
 
 def time_workload(d, device, steps, warmup, dist=None, soak_s=0.0, sampler=None, copies=0):
+    """Two timed regions over the same resident inputs: K steps through a plain plan (the
+    product path: the step value), then K steps through a plan that records events
+    around each launch (the per-kernel durations for the roofline)."""
     import torch
 
     import paged_head_latent_mla_b200 as M
@@ -273,14 +278,34 @@ def time_workload(d, device, steps, warmup, dist=None, soak_s=0.0, sampler=None,
     free, _ = torch.cuda.mem_get_info(device)
     while n_copies > 1 and n_copies * input_bytes(d) > 0.6 * free:
         n_copies -= 1
-    plan, step, out, lse, copies = make_runner(d, device, n_copies)
+    plan, step, out, lse, copies = make_runner(d, device, n_copies, timing=False)
+    tplan = M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=d.num_heads,
+                       page_size=d.page_size, num_pages=d.num_pages, sm_scale=d.sm_scale, causal=d.causal,
+                       debug_flags=M.MLA_DEBUG_KERNEL_TIMING)
+    lib = M.load_library()
+    import ctypes
+    stream = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    targs = [(tplan.handle, ctypes.c_void_p(qn.data_ptr()), ctypes.c_void_p(qp.data_ptr()),
+              ctypes.c_void_p(c.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+              ctypes.c_void_p(lse.data_ptr() if lse is not None else 0), stream) for (qn, qp, c) in copies]
+    tstate = {"i": 0}
+
+    def tstep():
+        a_ = targs[tstate["i"] % len(targs)]
+        tstate["i"] += 1
+        st_ = lib.mla_run(*a_)
+        if st_ != 0:
+            raise M.MlaError(st_, "mla_run")
+
     info = M.mla_plan_get_info(plan)
     for _ in range(warmup):
         step()
+        tstep()
     torch.cuda.synchronize(device)
-    st = M.mla_plan_check(plan)
-    if st != 0:
-        raise M.MlaError(st, "warm-up")
+    for pl in (plan, tplan):
+        st = M.mla_plan_check(pl)
+        if st != 0:
+            raise M.MlaError(st, "warm-up")
     if sampler is not None:
         sampler.start()
     if soak_s > 0:  # untimed: lets the clock sampler see the GPU under this load
@@ -301,16 +326,22 @@ def time_workload(d, device, steps, warmup, dist=None, soak_s=0.0, sampler=None,
     torch.cuda.synchronize(device)
     if dist is not None:
         dist.barrier()
-    clocks = sampler.stop() if sampler is not None else None
     ms = e0.elapsed_time(e1)
-    attn_ms, merge_ms = M.mla_plan_kernel_times(plan, capacity=min(steps, 256))
-    st = M.mla_plan_check(plan)
-    if st != 0:
-        raise M.MlaError(st, "timed steps")
+    # second region: per-kernel durations (events between the launches)
+    for _ in range(steps):
+        tstep()
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop() if sampler is not None else None
+    attn_ms, merge_ms = M.mla_plan_kernel_times(tplan, capacity=min(steps, 256))
+    for pl in (plan, tplan):
+        st = M.mla_plan_check(pl)
+        if st != 0:
+            raise M.MlaError(st, "timed steps")
     res = {"ms_total": ms, "ms_per_step": ms / steps, "attn_ms": float(attn_ms.mean()),
            "merge_ms": float(merge_ms.mean()), "info": info, "n_copies": n_copies, "clocks": clocks,
            "launches": steps * (1 + (1 if info["num_merge"] > 0 else 0))}
     plan.destroy()
+    tplan.destroy()
     del copies, out, lse
     torch.cuda.empty_cache()
     return res

@@ -10,6 +10,7 @@
 #include <limits>
 #include <mutex>
 #include <new>
+#include <vector>
 
 #include "mla_internal.h"
 
@@ -33,6 +34,7 @@ struct mla_plan_s {
   int32_t* d_kv_indices = nullptr;
   uint8_t* d_ws = nullptr;  // [partials][128][512] bf16 o, then [partials][128] fp32 lse
   void* h_staging = nullptr;
+  size_t blob_cap = 0, ws_cap = 0, staging_cap = 0;  // capacities of the pooled buffers
   cudaEvent_t ev_last = nullptr;
   // kernel timing ring (MLA_DEBUG_KERNEL_TIMING): 3 events per run
   static constexpr int kRing = 256;
@@ -44,9 +46,86 @@ namespace {
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Buffers of destroyed plans are kept for reuse, so that a caller that plans every step
+// (a serving loop whose batch changes each step) allocates nothing once the pool is
+// warm: cudaMalloc, cudaMallocHost and their frees synchronise and cost milliseconds.
+// Device buffers are keyed by device, pinned host buffers are not; capacities are powers
+// of two from 64 KB up, and at most kPoolKeep buffers of each kind and device are kept.
+enum PoolKind { kPoolDevice = 0, kPoolPinned = 1 };
+struct PoolEntry {
+  void* ptr;
+  size_t cap;
+  int device;
+  int kind;
+};
+std::mutex g_pool_mutex;
+std::vector<PoolEntry>* g_pool = new std::vector<PoolEntry>();  // never destroyed: usable during exit
+constexpr int kPoolKeep = 8;
+
+void* pool_take(int kind, int device, size_t bytes, size_t* cap) {
+  {
+    std::lock_guard<std::mutex> lock(g_pool_mutex);
+    int best = -1;
+    for (int i = 0; i < static_cast<int>(g_pool->size()); ++i) {
+      const PoolEntry& e = (*g_pool)[i];
+      if (e.kind == kind && (kind == kPoolPinned || e.device == device) && e.cap >= bytes &&
+          (best < 0 || e.cap < (*g_pool)[best].cap))
+        best = i;
+    }
+    if (best >= 0) {
+      void* ptr = (*g_pool)[best].ptr;
+      *cap = (*g_pool)[best].cap;
+      g_pool->erase(g_pool->begin() + best);
+      return ptr;
+    }
+  }
+  size_t c = size_t(64) << 10;
+  while (c < bytes) c <<= 1;
+  void* ptr = nullptr;
+  const cudaError_t e = kind == kPoolDevice ? cudaMalloc(&ptr, c) : cudaMallocHost(&ptr, c);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  *cap = c;
+  return ptr;
+}
+
+void pool_give(int kind, int device, void* ptr, size_t cap) {
+  if (!ptr) return;
+  PoolEntry evict{nullptr, 0, device, kind};
+  {
+    std::lock_guard<std::mutex> lock(g_pool_mutex);
+    g_pool->push_back(PoolEntry{ptr, cap, device, kind});
+    int n = 0, smallest = -1;
+    for (int i = 0; i < static_cast<int>(g_pool->size()); ++i) {
+      const PoolEntry& e = (*g_pool)[i];
+      if (e.kind != kind || (kind == kPoolDevice && e.device != device)) continue;
+      ++n;
+      if (smallest < 0 || e.cap < (*g_pool)[smallest].cap) smallest = i;
+    }
+    if (n > kPoolKeep) {
+      evict = (*g_pool)[smallest];
+      g_pool->erase(g_pool->begin() + smallest);
+    }
+  }
+  if (evict.ptr) {
+    if (evict.kind == kPoolDevice) {
+      int cur = -1;
+      cudaGetDevice(&cur);
+      cudaSetDevice(evict.device);
+      cudaFree(evict.ptr);
+      cudaSetDevice(cur);
+    } else {
+      cudaFreeHost(evict.ptr);
+    }
+  }
+}
+
 void free_plan(mla_plan_s* p) {
   if (!p) return;
   if (!p->host_only) {
+    // the buffers may still be in use by this plan's last launches
     if (p->ev_last) {
       cudaEventSynchronize(p->ev_last);
       cudaEventDestroy(p->ev_last);
@@ -56,9 +135,9 @@ void free_plan(mla_plan_s* p) {
         if (p->ring[i]) cudaEventDestroy(p->ring[i]);
       delete[] p->ring;
     }
-    if (p->d_blob) cudaFree(p->d_blob);
-    if (p->d_ws) cudaFree(p->d_ws);
-    if (p->h_staging) cudaFreeHost(p->h_staging);
+    pool_give(kPoolDevice, p->device, p->d_blob, p->blob_cap);
+    pool_give(kPoolDevice, p->device, p->d_ws, p->ws_cap);
+    pool_give(kPoolPinned, -1, p->h_staging, p->staging_cap);
   }
   delete p;
 }
@@ -123,8 +202,10 @@ mla_status mla_plan(const mla_dims* dims, int32_t batch, const int32_t* qo_indpt
   const size_t off_idx = align_up(off_merge + sizeof(MergeItem) * p->layout.merge.size(), 256);
   const size_t blob = align_up(off_idx + sizeof(int32_t) * n_idx, 256);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMalloc(&p->d_blob, blob) != cudaSuccess) { cudaGetLastError(); free_plan(p); return MLA_ERR_OUT_OF_MEMORY; }
-  if (cudaMallocHost(&p->h_staging, blob) != cudaSuccess) { cudaGetLastError(); free_plan(p); return MLA_ERR_OUT_OF_MEMORY; }
+  p->d_blob = pool_take(kPoolDevice, p->device, blob, &p->blob_cap);
+  if (!p->d_blob) { free_plan(p); return MLA_ERR_OUT_OF_MEMORY; }
+  p->h_staging = pool_take(kPoolPinned, -1, blob, &p->staging_cap);
+  if (!p->h_staging) { free_plan(p); return MLA_ERR_OUT_OF_MEMORY; }
   uint8_t* h = static_cast<uint8_t*>(p->h_staging);
   std::memset(h, 0, off_work);
   if (!p->layout.work.empty()) std::memcpy(h + off_work, p->layout.work.data(), sizeof(WorkItem) * p->layout.work.size());
@@ -138,7 +219,8 @@ mla_status mla_plan(const mla_dims* dims, int32_t batch, const int32_t* qo_indpt
   p->d_kv_indices = reinterpret_cast<int32_t*>(d + off_idx);
   if (p->layout.num_partials > 0) {
     const size_t ws = static_cast<size_t>(p->layout.num_partials) * kPartialBytes;
-    if (cudaMalloc(reinterpret_cast<void**>(&p->d_ws), ws) != cudaSuccess) { cudaGetLastError(); free_plan(p); return MLA_ERR_OUT_OF_MEMORY; }
+    p->d_ws = static_cast<uint8_t*>(pool_take(kPoolDevice, p->device, ws, &p->ws_cap));
+    if (!p->d_ws) { free_plan(p); return MLA_ERR_OUT_OF_MEMORY; }
   }
   if (p->opts.debug_flags & MLA_DEBUG_KERNEL_TIMING) {
     p->ring = new (std::nothrow) cudaEvent_t[3 * mla_plan_s::kRing]();
