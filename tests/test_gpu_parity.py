@@ -193,3 +193,50 @@ def test_full_size_config_sampled(name):
     assert np.isfinite(out).all()
     # properties that hold at any size: every lse finite (every query sees >= 1 key here)
     assert np.isfinite(lse).all()
+
+
+def test_pooled_plan_buffers_reused_across_shapes():
+    """mla_plan takes its device blob, split-KV workspace and pinned staging from a pool
+    that mla_plan_destroy refills.  Alternate plans of different sizes (so a plan often
+    receives a buffer that still holds another plan's work list or partials), keep two
+    plans alive at once (they must not share a buffer), and check every result."""
+    dev = torch.device("cuda:0")
+    cases = [make_custom([1, 1, 2], [9000, 300, 4100], 128, 64, seed=61),       # split partials
+             make_custom([3, 0, 1], [40, 7, 1300], 32, 16, seed=62),            # small, unsplit
+             make_custom([1] * 6, [5000 + 700 * i for i in range(6)], 64, 32, seed=63)]
+
+    def plan_of(d, split):
+        return M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=d.num_heads,
+                          page_size=d.page_size, num_pages=d.num_pages, sm_scale=d.sm_scale, causal=d.causal,
+                          split_keys=split, wait_timeout_ns=TEST_TIMEOUT_NS)
+
+    refs = [O.mla_attention(d.q_nope, d.q_pe, d.cache, d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len,
+                            d.page_size, d.sm_scale, causal=d.causal) for d in cases]
+    inputs = [(d.q_nope.to(dev), d.q_pe.to(dev), d.cache.to(dev)) for d in cases]
+
+    def check(i, out, lse):
+        ro, rl = refs[i]
+        o = out.float().cpu().numpy()
+        assert (np.abs(o - ro) <= OUT_ATOL + OUT_RTOL * np.abs(ro)).all()
+        gl = lse.cpu().numpy()
+        inf = np.isneginf(rl)
+        assert np.array_equal(inf, np.isneginf(gl))
+        if (~inf).any():
+            assert np.abs(gl[~inf] - rl[~inf]).max() <= LSE_ATOL
+
+    for rnd, order in enumerate(([0, 1, 2], [2, 0, 1], [1, 2, 0])):
+        for i in order:
+            plan = plan_of(cases[i], 128 if rnd % 2 == 0 else 0)
+            out, lse = M.mla_run(plan, *inputs[i], return_lse=True)
+            assert M.mla_plan_check(plan) == M.MLA_OK
+            plan.destroy()
+            check(i, out, lse)
+    # two live plans at once
+    a, b = plan_of(cases[0], 192), plan_of(cases[2], 128)
+    oa, la = M.mla_run(a, *inputs[0], return_lse=True)
+    ob, lb = M.mla_run(b, *inputs[2], return_lse=True)
+    assert M.mla_plan_check(a) == M.MLA_OK and M.mla_plan_check(b) == M.MLA_OK
+    check(0, oa, la)
+    check(2, ob, lb)
+    a.destroy()
+    b.destroy()
