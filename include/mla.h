@@ -74,6 +74,33 @@ typedef struct {
   int32_t host_only;        /* 1: build the work lists on the host only, touching no
                                CUDA API (for inspecting a plan on a machine without a
                                GPU); such a plan can be described but not run         */
+  /* Graph bucket (FlashInferMLAWrapper: use_cuda_graph with a batch_size fixed for the
+   * wrapper's life; base page: captured_page_capacity).  When graph_max_tokens > 0 the
+   * plan is a GRAPH PLAN: its device buffers and the launch shapes of mla_run and
+   * mla_append_kv are fixed for a bucket of at most graph_max_batch rows,
+   * graph_max_tokens query tokens and graph_max_page_ids page ids, so that a CUDA graph
+   * captured around mla_run replays correctly after mla_plan_update has re-planned the
+   * plan in place for another step of the bucket.  Unused launch slots are empty work
+   * items that return at once.  Every per-token buffer given to a graph plan (q_nope,
+   * q_pe, out, lse, kv_new) holds graph_max_tokens tokens; a step's T tokens are its
+   * first T.  All three bounds must be > 0 together.                                  */
+  int32_t graph_max_batch;
+  int32_t graph_max_tokens;
+  int32_t graph_max_page_ids;
+  /* 1: a CONTEXT-ONLY plan (FlashInferMLAManager.kv_len_buf): each row's queries attend
+   * only the row's stored context, keys j < c_b = k_b - q_b, all of which precede every
+   * query, so no causal mask applies; mla_plan_describe's kv_len reports c_b.  The page
+   * tables still cover the step's own q_b entries (mla_append_kv writes them at
+   * positions c_b + i).  Requires k_b >= q_b on every row.  The caller merges the
+   * result with an attention over the step's own tokens (mla_merge_state).          */
+  int32_t context_only;
+  /* 1: SHARED-PREFIX CASCADE.  Consecutive rows whose page lists begin with the same
+   * page ids (base page: captured_page_capacity, "rows that matched one cached prefix
+   * all name its pages") attend that shared prefix together: one work item per 128
+   * query rows of the whole group covers the prefix keys, its partial results are
+   * merged by log-sum-exp with each row's own suffix.  Applies where the shared prefix
+   * spans at least MLA_KEY_TILE keys and every query of the group sees all of it.    */
+  int32_t cascade;
 } mla_plan_options;
 
 /* Keys per tile of the attention kernel: work items start on multiples of it. */
@@ -91,7 +118,12 @@ typedef struct {
   int32_t num_merge;       /* query tiles whose keys were split                       */
   int32_t num_partials;    /* partial results the merge kernel combines               */
   int32_t num_sms;         /* SMs the plan was balanced for                           */
-  int64_t workspace_bytes; /* plan-owned split-KV workspace                           */
+  int64_t workspace_bytes; /* split-KV workspace in use                               */
+  int32_t num_merge_refs;  /* entries of the merge reference list                     */
+  int32_t num_cascade;     /* work items that attend a shared prefix for a row group  */
+  int32_t graph;           /* 1 for a graph plan                                      */
+  int32_t work_capacity;   /* launch slots of the attention grid (num_work unless a
+                              graph plan)                                             */
 } mla_plan_info;
 
 typedef struct mla_plan_s* mla_plan_t; /* opaque ("immutable and opaque to runner":
@@ -147,17 +179,77 @@ mla_status mla_plan_check(mla_plan_t plan);
 mla_status mla_plan_get_info(mla_plan_t plan, mla_plan_info* info);
 
 /* Copy the plan's bookkeeping to host arrays (each may be NULL):
- *   kv_len [batch]                      keys per row, k_b
+ *   kv_len [batch]                      keys per row: k_b, or c_b = k_b - q_b for a
+ *                                       context-only plan
  *   work   [num_work * MLA_WORK_FIELDS] one record per work item:
  *     { q_row0, n_rows, page_base, kv_len, key_begin, key_end, diag_base, partial }
- *     q_row0 = first (token * H + head) row of the 128-row query tile; n_rows valid
- *     rows; page_base = kv_indptr of the row; keys [key_begin, key_end) of the tile;
+ *     q_row0 = first (token * H + head) row of the query tile, n_rows its rows (at most
+ *     128; a cascade item's rows may span several batch rows of one group, every other
+ *     item's lie in one row); page_base = the kv_indptr entry whose pages the item
+ *     reads; kv_len = keys addressable from there; keys [key_begin, key_end);
  *     row r of the tile sees keys < clamp(diag_base + r / H + 1, 0, kv_len);
- *     partial = -1 (written straight to out/lse) or the workspace slot.
- *   merge  [num_merge * MLA_MERGE_FIELDS] { q_row0, n_rows, first_partial, n_partials } */
+ *     partial = -1 (written straight to out/lse) or the first workspace row of the
+ *     item's partial result (its row r lands in workspace row partial + r).
+ *   merge  [num_merge * MLA_MERGE_FIELDS] { q_row0, n_rows, first_ref, n_refs }: output
+ *     rows [q_row0, q_row0 + n_rows) combine the n_refs partial results whose row 0 is
+ *     workspace row refs[first_ref + i].
+ *   refs   [num_merge_refs]             the merge reference list. */
 #define MLA_WORK_FIELDS 8
 #define MLA_MERGE_FIELDS 4
-mla_status mla_plan_describe(mla_plan_t plan, int32_t* kv_len, int32_t* work, int32_t* merge);
+mla_status mla_plan_describe(mla_plan_t plan, int32_t* kv_len, int32_t* work, int32_t* merge, int32_t* refs);
+
+/* Re-plan a plan for another step, in place (base page: PlanCacheKey, "when it is
+ * unchanged between steps the re-plan is skippable"; FlashInferMLAWrapper.plan).
+ * Arguments as for mla_plan; dims, causal and options stay those of the plan.
+ *   *reused (may be NULL) receives 1 when the tables equal those of the plan's current
+ *   step (same batch, qo_indptr, kv_indptr, kv_indices and last_page_len): nothing is
+ *   planned or uploaded.  Otherwise 0: the plan is rebuilt and its device lists are
+ *   rewritten by an upload enqueued on `stream`, so runs enqueued on that stream
+ *   before the call see the old step and runs after it the new one.
+ * A graph plan keeps every device address and launch shape: a CUDA graph that captured
+ * mla_run (or mla_append_kv) on it replays the new step.  The step must fit the bucket
+ * (batch, tokens and page ids within the graph bounds), else INVALID_ARGUMENT and the
+ * plan is unchanged.  Other plans may grow their buffers (waiting for their last run
+ * first when they do).  The host staging is double-buffered: the call waits only for
+ * the upload of two updates ago, so the host may run one step ahead of the GPU
+ * (FlashInferMLAManager.force_double_buffer describes the race this avoids).
+ * Errors: INVALID_ARGUMENT, OUT_OF_MEMORY, CUDA; on error the plan still describes and
+ * runs its previous step. */
+mla_status mla_plan_update(mla_plan_t plan, int32_t batch, const int32_t* qo_indptr, const int32_t* kv_indptr,
+                           const int32_t* kv_indices, const int32_t* last_page_len, void* stream,
+                           int32_t* reused);
+
+/* Write the step's latent rows into their cache slots (base page: AttentionManager
+ * .requires_kv_write, "a layer must write this step's K/V through the KV resource
+ * before calling run").  Token i of row b (t = qo_indptr[b] + i) is key position
+ * k_b - q_b + i of its row, i.e. slot (k_b - q_b + i) mod page_size of page
+ * kv_indices[kv_indptr[b] + (k_b - q_b + i) / page_size]:
+ *   kv_new  device bf16 [T][576] ([ckv | kpe] per token), contiguous, 16-byte aligned
+ *   cache   device bf16 [num_pages][page_size][576] (written at those slots only)
+ * One launch, no allocation, no synchronisation.  Two tokens naming the same slot (a
+ * page listed twice) leave one of the two rows there.  Errors: INVALID_ARGUMENT (NULL
+ * or misaligned pointer, or a row with q_b > k_b, whose tokens have no slots), CUDA. */
+mla_status mla_append_kv(mla_plan_t plan, const void* kv_new, void* cache, void* stream);
+
+/* mla_append_kv followed by mla_run, as one enqueue: the attention launch is a
+ * programmatic dependent of the append launch, so its set-up (barriers, tensor memory,
+ * query tiles) overlaps the append and only its key loads wait for the append's
+ * writes.  Arguments and errors as for the two calls. */
+mla_status mla_run_append(mla_plan_t plan, const void* q_nope, const void* q_pe, const void* kv_new, void* cache,
+                          void* out, float* lse, void* stream);
+
+/* Merge two attention states over disjoint key sets by their log-sum-exps
+ * (FlashInferMLAManager.run: "the natural log-sum-exp of the scores ... for merging with
+ * another key segment"):
+ *   M = max(lse_a, lse_b);  w_x = exp(lse_x - M);
+ *   out = (w_a out_a + w_b out_b) / (w_a + w_b);  lse = M + ln(w_a + w_b)
+ * with a state whose lse is -inf contributing nothing (both -inf: out = 0, lse = -inf).
+ *   out_a, out_b, out   device bf16 [rows][512], 16-byte aligned (out may alias either)
+ *   lse_a, lse_b        device fp32 [rows]
+ *   lse                 device fp32 [rows] or NULL
+ * Errors: INVALID_ARGUMENT (NULL or misaligned pointer, rows < 0), CUDA. */
+mla_status mla_merge_state(const void* out_a, const float* lse_a, const void* out_b, const float* lse_b, void* out,
+                           float* lse, int64_t rows, void* stream);
 
 /* Kernel durations of the plan's most recent runs, for plans made with
  * MLA_DEBUG_KERNEL_TIMING: each mla_run records events on its stream before the

@@ -160,6 +160,7 @@ def mla_attention(
     sm_scale: float,
     causal: bool = True,
     tokens=None,
+    context_only: bool = False,
 ):
     """Paged absorbed-MLA attention, plain definition in float64.
 
@@ -167,6 +168,12 @@ def mla_attention(
     returns out [T, H, 512] and lse [T, H] (natural log).  With ``tokens`` (an
     iterable of global token indices) only those tokens are computed; the other
     entries of the result are NaN.
+
+    ``context_only``: every query of row b attends exactly the row's stored context,
+    keys ``j < k_b - q_b`` (flashinfer_mla page, ``FlashInferMLAManager.kv_len_buf``:
+    the planned length of a context-only row is its stored context, where its queries
+    start); those keys precede every query, so no mask applies.  A row with
+    ``q_b > k_b`` has no such context and is rejected.
     """
     qn = _f64(q_nope)
     qp = _f64(q_pe)
@@ -188,13 +195,17 @@ def mla_attention(
         if want is not None and not any(t in want for t in range(t0, t1)):
             continue
         k_b = int(k_all[b])
-        keys = gather_row_keys(cache, kv_indptr, kv_indices, page_size, b, k_b)
         q_b = t1 - t0
+        if context_only:
+            if k_b < q_b:
+                raise ValueError(f"row {b}: {q_b} queries but only {k_b} keys (no stored context)")
+            k_b -= q_b
+        keys = gather_row_keys(cache, kv_indptr, kv_indices, page_size, b, k_b)
         for i in range(q_b):
             t = t0 + i
             if want is not None and t not in want:
                 continue
-            vis = visible_keys(k_b, q_b, i, causal)
+            vis = k_b if context_only else visible_keys(k_b, q_b, i, causal)
             out[t], lse[t] = attend_one(q_full[t], keys, vis, sm_scale)
     return out, lse
 
@@ -236,3 +247,29 @@ def merge_many(outs, lses):
         lse = m_safe + np.log(z)
     empty = z == 0
     return np.where(empty[..., None], 0.0, out), np.where(empty, -np.inf, lse)
+
+
+def append_latent(cache, kv_new, qo_indptr, kv_indptr, kv_indices, last_page_len, page_size: int):
+    """The step's latent rows written into their cache slots (base page,
+    ``AttentionManager.requires_kv_write``: the layer writes the step's K/V before the
+    attention runs, so the row's keys end with its own tokens).
+
+    Token i of row b (global token ``qo_indptr[b] + i``) is logical key
+    ``k_b - q_b + i`` of its row; ``kv_new [T, 576]`` row t is stored at that key's
+    (page, slot).  Returns a float64 copy of ``cache`` with those rows replaced, in
+    token order (a later token wins where two name the same slot).  A row with
+    ``q_b > k_b`` has no slot for its first tokens and is rejected.
+    """
+    out = _f64(cache).copy()
+    new = _f64(kv_new)
+    qo_indptr = _i64(qo_indptr)
+    k_all = kv_lengths(kv_indptr, last_page_len, page_size)
+    for b in range(len(qo_indptr) - 1):
+        t0, t1 = int(qo_indptr[b]), int(qo_indptr[b + 1])
+        q_b, k_b = t1 - t0, int(k_all[b])
+        if q_b > k_b:
+            raise ValueError(f"row {b}: {q_b} new tokens but only {k_b} keys in its pages")
+        for i in range(q_b):
+            page, slot = key_location(kv_indptr, kv_indices, page_size, b, k_b - q_b + i)
+            out[page, slot] = new[t0 + i]
+    return out

@@ -6,7 +6,8 @@ runs in the library's CUDA kernels.  If the library is missing the calls raise; 
 is no other implementation to fall back to.
 
 Names follow the C ABI in ``include/mla.h``: ``mla_supports``, ``mla_plan``,
-``mla_run``, ``mla_plan_check``, ``mla_plan_get_info``, ``mla_plan_describe``,
+``mla_plan_update``, ``mla_run``, ``mla_append_kv``, ``mla_run_append``,
+``mla_merge_state``, ``mla_plan_check``, ``mla_plan_get_info``, ``mla_plan_describe``,
 ``mla_plan_kernel_times``, ``mla_run_noalloc``, ``mla_plan_destroy``,
 ``mla_status_string``.
 """
@@ -39,7 +40,11 @@ ROPE_DIM = 64
 EXPORTED = (
     "mla_supports",
     "mla_plan",
+    "mla_plan_update",
     "mla_run",
+    "mla_append_kv",
+    "mla_run_append",
+    "mla_merge_state",
     "mla_plan_check",
     "mla_plan_get_info",
     "mla_plan_describe",
@@ -74,6 +79,11 @@ class _Options(ctypes.Structure):
         ("wait_timeout_ns", ctypes.c_uint64),
         ("debug_flags", ctypes.c_int32),
         ("host_only", ctypes.c_int32),
+        ("graph_max_batch", ctypes.c_int32),
+        ("graph_max_tokens", ctypes.c_int32),
+        ("graph_max_page_ids", ctypes.c_int32),
+        ("context_only", ctypes.c_int32),
+        ("cascade", ctypes.c_int32),
     ]
 
 
@@ -86,6 +96,10 @@ class _Info(ctypes.Structure):
         ("num_partials", ctypes.c_int32),
         ("num_sms", ctypes.c_int32),
         ("workspace_bytes", ctypes.c_int64),
+        ("num_merge_refs", ctypes.c_int32),
+        ("num_cascade", ctypes.c_int32),
+        ("graph", ctypes.c_int32),
+        ("work_capacity", ctypes.c_int32),
     ]
 
 
@@ -111,11 +125,19 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_plan.restype = ctypes.c_int
     lib.mla_run.argtypes = [vp, vp, vp, vp, vp, vp, vp]
     lib.mla_run.restype = ctypes.c_int
+    lib.mla_plan_update.argtypes = [vp, ctypes.c_int32, i32p, i32p, i32p, i32p, vp, i32p]
+    lib.mla_plan_update.restype = ctypes.c_int
+    lib.mla_append_kv.argtypes = [vp, vp, vp, vp]
+    lib.mla_append_kv.restype = ctypes.c_int
+    lib.mla_run_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.mla_run_append.restype = ctypes.c_int
+    lib.mla_merge_state.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_int64, vp]
+    lib.mla_merge_state.restype = ctypes.c_int
     lib.mla_plan_check.argtypes = [vp]
     lib.mla_plan_check.restype = ctypes.c_int
     lib.mla_plan_get_info.argtypes = [vp, ctypes.POINTER(_Info)]
     lib.mla_plan_get_info.restype = ctypes.c_int
-    lib.mla_plan_describe.argtypes = [vp, i32p, i32p, i32p]
+    lib.mla_plan_describe.argtypes = [vp, i32p, i32p, i32p, i32p]
     lib.mla_plan_describe.restype = ctypes.c_int
     fp = ctypes.POINTER(ctypes.c_float)
     lib.mla_plan_kernel_times.argtypes = [vp, ctypes.c_int32, fp, fp, i32p]
@@ -162,11 +184,18 @@ def mla_supports(kv_lora_rank: int, rope_dim: int, num_heads: int, page_size: in
 class MlaPlan:
     """Owns one C plan handle (``mla_plan_t``); destroyed with the object."""
 
-    def __init__(self, handle: int, batch: int, num_heads: int, total_tokens: int):
+    def __init__(self, handle: int, batch: int, num_heads: int, total_tokens: int, graph_max_tokens: int = 0):
         self._h = ctypes.c_void_p(handle)
         self.batch = batch
         self.num_heads = num_heads
         self.total_tokens = total_tokens
+        # a graph plan's per-token buffers hold graph_max_tokens tokens
+        self.graph_max_tokens = graph_max_tokens
+
+    @property
+    def token_capacity(self) -> int:
+        """Tokens every per-token buffer passed with this plan must hold."""
+        return self.graph_max_tokens if self.graph_max_tokens > 0 else self.total_tokens
 
     @property
     def handle(self) -> ctypes.c_void_p:
@@ -189,8 +218,13 @@ class MlaPlan:
 def mla_plan(qo_indptr, kv_indptr, kv_indices, last_page_len, *, num_heads: int, page_size: int, num_pages: int,
              sm_scale: float, causal: bool = True, kv_lora_rank: int = KV_LORA_RANK, rope_dim: int = ROPE_DIM,
              split_keys: int = 0, num_sms: int = 0, wait_timeout_ns: int = 0, debug_flags: int = 0,
-             host_only: bool = False, stream=None) -> MlaPlan:
-    """Plan one step from host page tables (``mla_plan``)."""
+             host_only: bool = False, graph_max_batch: int = 0, graph_max_tokens: int = 0,
+             graph_max_page_ids: int = 0, context_only: bool = False, cascade: bool = False,
+             stream=None) -> MlaPlan:
+    """Plan one step from host page tables (``mla_plan``).  ``graph_max_*`` make a graph
+    plan for a bucket (fixed device buffers and launch shapes, re-planned in place by
+    ``mla_plan_update``); ``context_only`` attends only each row's stored context;
+    ``cascade`` attends prefixes shared by consecutive rows once per group."""
     lib = load_library()
     qo = _i32(qo_indptr)
     kvp = _i32(kv_indptr)
@@ -202,7 +236,8 @@ def mla_plan(qo_indptr, kv_indptr, kv_indices, last_page_len, *, num_heads: int,
     if len(kvi) < int(kvp[-1]):
         raise MlaError(MLA_ERR_INVALID_ARGUMENT, "mla_plan: kv_indices shorter than kv_indptr[-1]")
     dims = _Dims(num_heads, kv_lora_rank, rope_dim, page_size, num_pages, sm_scale)
-    opts = _Options(split_keys, num_sms, wait_timeout_ns, debug_flags, 1 if host_only else 0)
+    opts = _Options(split_keys, num_sms, wait_timeout_ns, debug_flags, 1 if host_only else 0, graph_max_batch,
+                    graph_max_tokens, graph_max_page_ids, 1 if context_only else 0, 1 if cascade else 0)
     if stream is None and not host_only:
         import torch
 
@@ -213,7 +248,34 @@ def mla_plan(qo_indptr, kv_indptr, kv_indices, last_page_len, *, num_heads: int,
                       1 if causal else 0, ctypes.c_void_p(stream or 0), ctypes.byref(opts), ctypes.byref(out))
     if st != MLA_OK:
         raise MlaError(st, "mla_plan")
-    return MlaPlan(out.value, batch, num_heads, int(qo[-1]))
+    return MlaPlan(out.value, batch, num_heads, int(qo[-1]), graph_max_tokens if graph_max_tokens > 0 else 0)
+
+
+def mla_plan_update(plan: MlaPlan, qo_indptr, kv_indptr, kv_indices, last_page_len, stream=None) -> bool:
+    """Re-plan ``plan`` in place for another step (``mla_plan_update``).  Returns True
+    when the tables equal the plan's current step and nothing was done."""
+    lib = load_library()
+    qo = _i32(qo_indptr)
+    kvp = _i32(kv_indptr)
+    kvi = _i32(kv_indices)
+    last = _i32(last_page_len)
+    batch = len(qo) - 1
+    if batch < 0 or len(kvp) != batch + 1 or len(last) != batch or len(kvi) < int(kvp[-1]):
+        raise MlaError(MLA_ERR_INVALID_ARGUMENT, "mla_plan_update: table lengths")
+    if stream is None:
+        import torch
+
+        stream = torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else 0
+    kvi_arr = kvi if len(kvi) else np.zeros(1, dtype=np.int32)
+    last_arr = last if len(last) else np.zeros(1, dtype=np.int32)
+    reused = ctypes.c_int32(0)
+    st = lib.mla_plan_update(plan.handle, batch, _ptr(qo), _ptr(kvp), _ptr(kvi_arr), _ptr(last_arr),
+                             ctypes.c_void_p(stream or 0), ctypes.byref(reused))
+    if st != MLA_OK:
+        raise MlaError(st, "mla_plan_update")
+    plan.batch = batch
+    plan.total_tokens = int(qo[-1])
+    return bool(reused.value)
 
 
 def mla_plan_get_info(plan: MlaPlan) -> dict:
@@ -225,18 +287,21 @@ def mla_plan_get_info(plan: MlaPlan) -> dict:
 
 
 def mla_plan_describe(plan: MlaPlan) -> dict:
-    """kv_len [B], work [num_work, 8] and merge [num_merge, 4] as int32 arrays."""
+    """kv_len [B], work [num_work, 8], merge [num_merge, 4] and the merge reference list
+    refs [num_merge_refs] as int32 arrays."""
     info = mla_plan_get_info(plan)
     kv_len = np.zeros(max(1, info["batch"]), dtype=np.int32)
     work = np.zeros((max(1, info["num_work"]), WORK_FIELDS), dtype=np.int32)
     merge = np.zeros((max(1, info["num_merge"]), MERGE_FIELDS), dtype=np.int32)
-    st = load_library().mla_plan_describe(plan.handle, _ptr(kv_len), _ptr(work), _ptr(merge))
+    refs = np.zeros(max(1, info["num_merge_refs"]), dtype=np.int32)
+    st = load_library().mla_plan_describe(plan.handle, _ptr(kv_len), _ptr(work), _ptr(merge), _ptr(refs))
     if st != MLA_OK:
         raise MlaError(st, "mla_plan_describe")
     return {
         "kv_len": kv_len[: info["batch"]],
         "work": work[: info["num_work"]],
         "merge": merge[: info["num_merge"]],
+        "refs": refs[: info["num_merge_refs"]],
         "info": info,
     }
 
@@ -254,11 +319,14 @@ def _check_dev_tensor(t, name, dtype, shape):
         raise ValueError(f"{name} must be contiguous")
 
 
-def mla_run(plan: MlaPlan, q_nope, q_pe, cache, out=None, lse=None, return_lse: bool = False, stream=None):
-    """Run the planned attention (``mla_run``).  Returns ``out`` or ``(out, lse)``."""
+def mla_run(plan: MlaPlan, q_nope, q_pe, cache, out=None, lse=None, return_lse: bool = False, stream=None,
+            kv_new=None):
+    """Run the planned attention (``mla_run``).  Returns ``out`` or ``(out, lse)``.
+    With ``kv_new`` ([T, 576] bf16) the step's latent rows are first written into the
+    cache (``mla_run_append``)."""
     import torch
 
-    T, H = plan.total_tokens, plan.num_heads
+    T, H = plan.token_capacity, plan.num_heads
     _check_dev_tensor(q_nope, "q_nope", torch.bfloat16, (T, H, KV_LORA_RANK))
     _check_dev_tensor(q_pe, "q_pe", torch.bfloat16, (T, H, ROPE_DIM))
     if cache.dim() != 3 or cache.shape[-1] != KV_LORA_RANK + ROPE_DIM:
@@ -271,15 +339,73 @@ def mla_run(plan: MlaPlan, q_nope, q_pe, cache, out=None, lse=None, return_lse: 
         lse = torch.empty((T, H), dtype=torch.float32, device=q_nope.device)
     if lse is not None:
         _check_dev_tensor(lse, "lse", torch.float32, (T, H))
+    if kv_new is not None:
+        _check_dev_tensor(kv_new, "kv_new", torch.bfloat16, (T, KV_LORA_RANK + ROPE_DIM))
     if stream is None:
         stream = torch.cuda.current_stream(q_nope.device).cuda_stream
-    st = load_library().mla_run(plan.handle, ctypes.c_void_p(q_nope.data_ptr()), ctypes.c_void_p(q_pe.data_ptr()),
-                                ctypes.c_void_p(cache.data_ptr()), ctypes.c_void_p(out.data_ptr()),
-                                ctypes.c_void_p(lse.data_ptr() if lse is not None else 0),
-                                ctypes.c_void_p(stream or 0))
+    lib = load_library()
+    lse_p = ctypes.c_void_p(lse.data_ptr() if lse is not None else 0)
+    if kv_new is None:
+        st = lib.mla_run(plan.handle, ctypes.c_void_p(q_nope.data_ptr()), ctypes.c_void_p(q_pe.data_ptr()),
+                         ctypes.c_void_p(cache.data_ptr()), ctypes.c_void_p(out.data_ptr()), lse_p,
+                         ctypes.c_void_p(stream or 0))
+        what = "mla_run"
+    else:
+        st = lib.mla_run_append(plan.handle, ctypes.c_void_p(q_nope.data_ptr()), ctypes.c_void_p(q_pe.data_ptr()),
+                                ctypes.c_void_p(kv_new.data_ptr()), ctypes.c_void_p(cache.data_ptr()),
+                                ctypes.c_void_p(out.data_ptr()), lse_p, ctypes.c_void_p(stream or 0))
+        what = "mla_run_append"
     if st != MLA_OK:
-        raise MlaError(st, "mla_run")
+        raise MlaError(st, what)
     return (out, lse) if (return_lse or lse is not None) else out
+
+
+def mla_append_kv(plan: MlaPlan, kv_new, cache, stream=None) -> None:
+    """Write the step's latent rows ``kv_new`` [T, 576] into their cache slots
+    (``mla_append_kv``)."""
+    import torch
+
+    _check_dev_tensor(kv_new, "kv_new", torch.bfloat16, (plan.token_capacity, KV_LORA_RANK + ROPE_DIM))
+    if cache.dim() != 3 or cache.shape[-1] != KV_LORA_RANK + ROPE_DIM:
+        raise ValueError("cache must be [num_pages, page_size, 576]")
+    _check_dev_tensor(cache, "cache", torch.bfloat16, tuple(cache.shape))
+    if stream is None:
+        stream = torch.cuda.current_stream(kv_new.device).cuda_stream
+    st = load_library().mla_append_kv(plan.handle, ctypes.c_void_p(kv_new.data_ptr()),
+                                      ctypes.c_void_p(cache.data_ptr()), ctypes.c_void_p(stream or 0))
+    if st != MLA_OK:
+        raise MlaError(st, "mla_append_kv")
+
+
+def mla_merge_state(out_a, lse_a, out_b, lse_b, out=None, lse=None, stream=None):
+    """Merge two attention states over disjoint key sets by their log-sum-exps
+    (``mla_merge_state``).  ``out_*`` bf16 [..., 512], ``lse_*`` fp32 [...].  Returns
+    ``(out, lse)``; ``out`` may be ``out_a`` or ``out_b``."""
+    import torch
+
+    shape = tuple(out_a.shape)
+    if len(shape) < 1 or shape[-1] != KV_LORA_RANK:
+        raise ValueError("out_a must be [..., 512]")
+    _check_dev_tensor(out_a, "out_a", torch.bfloat16, shape)
+    _check_dev_tensor(out_b, "out_b", torch.bfloat16, shape)
+    _check_dev_tensor(lse_a, "lse_a", torch.float32, shape[:-1])
+    _check_dev_tensor(lse_b, "lse_b", torch.float32, shape[:-1])
+    if out is None:
+        out = torch.empty_like(out_a)
+    if lse is None:
+        lse = torch.empty_like(lse_a)
+    _check_dev_tensor(out, "out", torch.bfloat16, shape)
+    _check_dev_tensor(lse, "lse", torch.float32, shape[:-1])
+    if stream is None:
+        stream = torch.cuda.current_stream(out_a.device).cuda_stream
+    rows = int(np.prod(shape[:-1])) if len(shape) > 1 else 1
+    st = load_library().mla_merge_state(
+        ctypes.c_void_p(out_a.data_ptr()), ctypes.c_void_p(lse_a.data_ptr()), ctypes.c_void_p(out_b.data_ptr()),
+        ctypes.c_void_p(lse_b.data_ptr()), ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(lse.data_ptr()),
+        ctypes.c_int64(rows), ctypes.c_void_p(stream or 0))
+    if st != MLA_OK:
+        raise MlaError(st, "mla_merge_state")
+    return out, lse
 
 
 def mla_plan_kernel_times(plan: MlaPlan, capacity: int = 256):

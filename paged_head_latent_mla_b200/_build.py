@@ -13,7 +13,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmla_b200.so")
-SOURCES = ["api.cu", "mla_attn.cu", "plan.cpp", "noalloc.cu"]
+SOURCES = ["api.cu", "mla_attn.cu", "state_ops.cu", "plan.cpp", "noalloc.cu"]
 HEADERS = ["mla_internal.h", "mla_launch.h", "sm100_ptx.cuh"]
 
 

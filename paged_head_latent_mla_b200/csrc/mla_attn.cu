@@ -146,6 +146,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   // this grid to finish before reading anything.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const WorkItem w = p.work[blockIdx.x >> 1];
+  // An empty launch slot (graph plans launch a fixed grid): both CTAs of the pair read
+  // the same item and leave before touching any shared state.
+  if (w.n_rows <= 0) return;
   const int ntiles = w.key_end > w.key_begin ? (w.key_end - w.key_begin + kTileN - 1) / kTileN : 0;
 
   auto bar = [&](int i) -> uint32_t { return sb + kBar + 8u * i; };
@@ -228,6 +231,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       int last_issued[kStages];
 #pragma unroll
       for (int s2 = 0; s2 < kStages; ++s2) last_issued[s2] = -1;
+      // Launched as a programmatic dependent of a cache append, the key loads must see
+      // its writes: wait for that grid (a no-op for an ordinary launch).
+      asm volatile("griddepcontrol.wait;" ::: "memory");
       for (int j = 0; j < ntiles; ++j) {
         const int st = j % kStages;
         if (j >= kStages && !wait_warp(bar(bKVEmpty + st), ((j / kStages) - 1) & 1, kSiteProducer, false)) break;
@@ -548,7 +554,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         }
         __syncwarp();
         const int nrows = min(32, w.n_rows - 32 * q);  // rows of this warp inside the tile
-        uint8_t* base = part ? static_cast<uint8_t*>(p.ws_o) + static_cast<size_t>(w.partial) * kTileM * kCkv * 2
+        uint8_t* base = part ? static_cast<uint8_t*>(p.ws_o) + static_cast<size_t>(w.partial) * kCkv * 2
                              : static_cast<uint8_t*>(p.out) + static_cast<size_t>(w.q_row0) * kCkv * 2;
         for (int R = 0; R < nrows; ++R) {
           uint8_t* dst = base + (static_cast<size_t>(32 * q + R) * kCkv + 256 * rank) * 2;
@@ -559,7 +565,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           if (!part) {
             if (p.lse != nullptr) p.lse[w.q_row0 + r] = lse_nat;
           } else {
-            p.ws_lse[static_cast<size_t>(w.partial) * kTileM + r] = lse_nat;
+            p.ws_lse[static_cast<size_t>(w.partial) + r] = lse_nat;
           }
         }
       }
@@ -578,7 +584,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   cluster_wait();
 }
 
-// Combine the partials of split query tiles by their log-sum-exp:
+// Combine the partials of split (or cascaded) query tiles by their log-sum-exp:
 // M = max_i lse_i, out = sum_i e^{lse_i - M} o_i / sum_i e^{lse_i - M},
 // lse = M + ln sum_i e^{lse_i - M} (FlashInferMLAManager.run: merging key segments).
 // One warp per row; lane l owns columns [16l, 16l + 16), so every load and store of a
@@ -592,9 +598,10 @@ __global__ void __launch_bounds__(256) mla_merge_kernel(const MergeParams p) {
   const int r = ((blockIdx.x & 15) << 3) + warp;  // 8 rows (one per warp) per block
   if (r >= m.n_rows) return;
   const float neg_inf = -__int_as_float(0x7f800000);
-  const int n = m.n_partials;
+  const int n = m.n_refs;
+  const int32_t* refs = p.refs + m.first_ref;  // workspace row of each partial's row 0
   float M = neg_inf;
-  for (int i = lane; i < n; i += 32) M = fmaxf(M, p.ws_lse[static_cast<size_t>(m.first_partial + i) * kTileM + r]);
+  for (int i = lane; i < n; i += 32) M = fmaxf(M, p.ws_lse[static_cast<size_t>(refs[i]) + r]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   float acc[16];
@@ -605,8 +612,8 @@ __global__ void __launch_bounds__(256) mla_merge_kernel(const MergeParams p) {
     for (int i0 = 0; i0 < n; i0 += 32) {
       const int cnt = min(32, n - i0);
       // lane u holds the weight of partial i0 + u
-      const float wl =
-          lane < cnt ? __expf(p.ws_lse[static_cast<size_t>(m.first_partial + i0 + lane) * kTileM + r] - M) : 0.f;
+      const int ref_l = lane < cnt ? refs[i0 + lane] : 0;
+      const float wl = lane < cnt ? __expf(p.ws_lse[static_cast<size_t>(ref_l) + r] - M) : 0.f;
       z += wl;
       for (int k = 0; k < cnt; k += 4) {
         uint4 v[4][2];
@@ -614,10 +621,10 @@ __global__ void __launch_bounds__(256) mla_merge_kernel(const MergeParams p) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           wk[u] = __shfl_sync(0xffffffffu, wl, k + u);  // k + u <= 31
+          const int ref_u = __shfl_sync(0xffffffffu, ref_l, k + u);
           if (k + u < cnt) {
             const uint4* src = reinterpret_cast<const uint4*>(
-                static_cast<const uint8_t*>(p.ws_o) +
-                ((static_cast<size_t>(m.first_partial + i0 + k + u) * kTileM + r) * kCkv + 16 * lane) * 2);
+                static_cast<const uint8_t*>(p.ws_o) + ((static_cast<size_t>(ref_u) + r) * kCkv + 16 * lane) * 2);
             v[u][0] = src[0];
             v[u][1] = src[1];
           } else {
@@ -710,8 +717,22 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
       !encode_2d(&tm_kv, a.cache, a.cache_rows, kLatent, 64, br, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&tm_kpe, a.cache, a.cache_rows, kLatent, 32, br, CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
-  mla_attn_kernel<<<2 * a.num_work, attn::kThreads, attn::kSmemAlloc, stream>>>(tm_q, tm_qpe, tm_kv, tm_kpe, p);
-  return cudaGetLastError();
+  if (!a.wait_prior_grid) {
+    mla_attn_kernel<<<2 * a.num_work, attn::kThreads, attn::kSmemAlloc, stream>>>(tm_q, tm_qpe, tm_kv, tm_kpe, p);
+    return cudaGetLastError();
+  }
+  // Programmatic dependent of the append: set-up and query loads overlap it.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2u * static_cast<unsigned>(a.num_work));
+  cfg.blockDim = dim3(attn::kThreads);
+  cfg.dynamicSmemBytes = attn::kSmemAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mla_attn_kernel, tm_q, tm_qpe, tm_kv, tm_kpe, p);
 }
 
 cudaError_t launch_merge(const MergeParams& p, int num_merge, cudaStream_t stream) {

@@ -40,19 +40,42 @@ struct AttnLaunch {
   const void* cache;    // bf16 [cache_rows, 576]
   uint64_t rows;        // T * H
   uint64_t cache_rows;  // num_pages * page_size
-  int num_work;
+  int num_work;         // launch slots (CTA pairs)
+  bool wait_prior_grid; // launched as a programmatic dependent of the previous kernel
+                        // (an append): the key loads wait for that grid's writes
 };
 
 struct MergeParams {
   const MergeItem* merge;
+  const int32_t* refs;
   const void* ws_o;
   const float* ws_lse;
   void* out;
   float* lse;
 };
 
+// Latent-cache append: token t's row of src goes to cache row rows[t] (skipped if < 0).
+struct AppendParams {
+  const int32_t* rows;  // [tokens]
+  const void* src;      // bf16 [tokens, 576]
+  void* cache;          // bf16 [cache_rows, 576]
+};
+
+// Merge of two attention states by their log-sum-exps.
+struct MergeStateParams {
+  const void* out_a;
+  const float* lse_a;
+  const void* out_b;
+  const float* lse_b;
+  void* out;
+  float* lse;  // may be null
+  int64_t rows;
+};
+
 // cudaErrorInvalidValue when a tensor map cannot be encoded.
 cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream);
 cudaError_t launch_merge(const MergeParams& p, int num_merge, cudaStream_t stream);
+cudaError_t launch_append(const AppendParams& p, int num_tokens, cudaStream_t stream);
+cudaError_t launch_merge_state(const MergeStateParams& p, cudaStream_t stream);
 
 }  // namespace mla

@@ -38,15 +38,18 @@ constexpr int kMaxPageIds = 1 << 19;                // kv_indptr[batch]
 constexpr size_t kOffStatus = 0;
 constexpr size_t kOffWork = 256;
 constexpr size_t kOffMerge = kOffWork + sizeof(WorkItem) * kMaxWork;
-constexpr size_t kOffPages = kOffMerge + sizeof(MergeItem) * kMaxMerge;
+constexpr size_t kOffRefs = kOffMerge + sizeof(MergeItem) * kMaxMerge;
+constexpr size_t kOffPages = kOffRefs + sizeof(int32_t) * kMaxWork;
 constexpr size_t kOffPartials = (kOffPages + sizeof(int32_t) * kMaxPageIds + 255) / 256 * 256;
-constexpr int kMaxPartials = static_cast<int>((kScratchBytes - kOffPartials) / kPartialBytes);
-static_assert(kMaxPartials >= 32, "scratch too small for useful splitting");
+// workspace rows of split partial results (each partial takes its tile's rows)
+constexpr int kMaxWsRows = static_cast<int>((kScratchBytes - kOffPartials) / kWsRowBytes);
+static_assert(kMaxWsRows >= 32 * kTileM, "scratch too small for useful splitting");
 
 // Host-side planning buffers: static, so planning never touches the heap.  Calls that
 // overlap on the host would race on these, like they race on the device array.
 WorkItem g_work[kMaxWork];
 MergeItem g_merge[kMaxMerge];
+int32_t g_refs[kMaxWork];
 
 struct DeviceScratch {
   unsigned char* ptr = nullptr;
@@ -58,10 +61,10 @@ std::mutex g_dev_mutex;
 
 // Validate the tables and cut the work into g_work / g_merge without allocating.
 // Long key ranges are split into chunks of about (total tiles / SM pairs) tiles while
-// partial slots remain in the scratch array; the rest run unsplit.
+// workspace rows remain in the scratch array; the rest run unsplit.
 mla_status plan_fixed(const mla_dims& d, int32_t batch, const int32_t* qo, const int32_t* kvp,
                       const int32_t* kvi, const int32_t* last, bool causal, int num_sms, int* n_work,
-                      int* n_merge, int* n_partials, int32_t* total_tokens) {
+                      int* n_merge, int* n_refs, int* n_ws_rows, int32_t* total_tokens) {
   if (!shape_supported(d.kv_lora_rank, d.rope_dim, d.num_heads, d.page_size)) return MLA_ERR_UNSUPPORTED;
   if (batch < 0 || d.num_pages < 1 || !std::isfinite(d.sm_scale) || !(d.sm_scale > 0.f))
     return MLA_ERR_INVALID_ARGUMENT;
@@ -98,7 +101,7 @@ mla_status plan_fixed(const mla_dims& d, int32_t batch, const int32_t* qo, const
   const int units = std::max(1, num_sms / 2);
   const int64_t chunk = std::max<int64_t>(8, (total_tiles + units - 1) / units);
   // pass 2: emit (every tile still to come keeps at least one work slot)
-  int nw = 0, nm = 0, np = 0;
+  int nw = 0, nm = 0, nr = 0, rows_used = 0;
   int64_t tiles_left = n_tiles;
   for (int32_t b = 0; b < batch; ++b) {
     const int64_t n = kvp[b + 1] - kvp[b];
@@ -113,7 +116,7 @@ mla_status plan_fixed(const mla_dims& d, int32_t batch, const int32_t* qo, const
       const int32_t q_row0 = (qo[b] + tok0) * H;
       int32_t pieces = nt > chunk ? static_cast<int32_t>((nt + chunk - 1) / chunk) : 1;
       --tiles_left;
-      if (pieces > 1 && (np + pieces > kMaxPartials || nm >= kMaxMerge ||
+      if (pieces > 1 && (rows_used + pieces * ntok * H > kMaxWsRows || nm >= kMaxMerge ||
                          nw + pieces + tiles_left > kMaxWork))
         pieces = 1;  // no scratch left for partials: run this tile unsplit
       if (nw + pieces > kMaxWork) return MLA_ERR_INVALID_ARGUMENT;
@@ -121,12 +124,14 @@ mla_status plan_fixed(const mla_dims& d, int32_t batch, const int32_t* qo, const
         g_work[nw++] = WorkItem{q_row0, ntok * H, kvp[b], k, 0, vis_hi, diag, -1};
         continue;
       }
-      g_merge[nm++] = MergeItem{q_row0, ntok * H, np, pieces};
+      g_merge[nm++] = MergeItem{q_row0, ntok * H, nr, pieces};
       for (int32_t i = 0; i < pieces; ++i) {
         const int32_t lo = int32_t(int64_t(nt) * i / pieces), hi = int32_t(int64_t(nt) * (i + 1) / pieces);
-        g_work[nw++] = WorkItem{q_row0, ntok * H, kvp[b], k, lo * kTileN, std::min(hi * kTileN, vis_hi), diag, np + i};
+        g_refs[nr++] = rows_used;
+        g_work[nw++] =
+            WorkItem{q_row0, ntok * H, kvp[b], k, lo * kTileN, std::min(hi * kTileN, vis_hi), diag, rows_used};
+        rows_used += ntok * H;
       }
-      np += pieces;
     }
   }
   std::sort(g_work, g_work + nw, [](const WorkItem& a, const WorkItem& c) {
@@ -134,7 +139,8 @@ mla_status plan_fixed(const mla_dims& d, int32_t batch, const int32_t* qo, const
   });
   *n_work = nw;
   *n_merge = nm;
-  *n_partials = np;
+  *n_refs = nr;
+  *n_ws_rows = rows_used;
   *total_tokens = static_cast<int32_t>(T);
   return MLA_OK;
 }
@@ -172,10 +178,10 @@ extern "C" mla_status mla_run_noalloc(const mla_dims* dims, int32_t batch, const
   }
   unsigned char* scratch = g_dev[dev].ptr;
 
-  int n_work = 0, n_merge = 0, n_partials = 0;
+  int n_work = 0, n_merge = 0, n_refs = 0, n_ws_rows = 0;
   int32_t T = 0;
   mla_status st = plan_fixed(*dims, batch, qo_indptr, kv_indptr, kv_indices, last_page_len, causal != 0,
-                             g_dev[dev].num_sms, &n_work, &n_merge, &n_partials, &T);
+                             g_dev[dev].num_sms, &n_work, &n_merge, &n_refs, &n_ws_rows, &T);
   if (st != MLA_OK) return st;
   if (n_work == 0) return MLA_OK;
   if (!q_nope || !q_pe || !cache || !out) return MLA_ERR_INVALID_ARGUMENT;
@@ -194,6 +200,8 @@ extern "C" mla_status mla_run_noalloc(const mla_dims* dims, int32_t batch, const
           cudaSuccess ||
       (n_merge > 0 && cudaMemcpyAsync(scratch + kOffMerge, g_merge, sizeof(MergeItem) * n_merge,
                                       cudaMemcpyHostToDevice, s) != cudaSuccess) ||
+      (n_merge > 0 && cudaMemcpyAsync(scratch + kOffRefs, g_refs, sizeof(int32_t) * n_refs,
+                                      cudaMemcpyHostToDevice, s) != cudaSuccess) ||
       (n_idx > 0 && cudaMemcpyAsync(scratch + kOffPages, kv_indices, sizeof(int32_t) * n_idx,
                                     cudaMemcpyHostToDevice, s) != cudaSuccess)) {
     cudaGetLastError();
@@ -208,7 +216,7 @@ extern "C" mla_status mla_run_noalloc(const mla_dims* dims, int32_t batch, const
   ap.out = out;
   ap.lse = lse;
   ap.ws_o = partials;
-  ap.ws_lse = reinterpret_cast<float*>(partials + size_t(n_partials) * kPartialOBytes);
+  ap.ws_lse = reinterpret_cast<float*>(partials + size_t(n_ws_rows) * kWsRowOBytes);
   ap.status = reinterpret_cast<int32_t*>(scratch + kOffStatus);
   ap.scale_log2 = dims->sm_scale * 1.4426950408889634f;
   ap.num_heads = dims->num_heads;
@@ -221,9 +229,11 @@ extern "C" mla_status mla_run_noalloc(const mla_dims* dims, int32_t batch, const
   a.rows = uint64_t(T) * dims->num_heads;
   a.cache_rows = uint64_t(dims->num_pages) * dims->page_size;
   a.num_work = n_work;
+  a.wait_prior_grid = false;
   if (launch_attention(a, s) != cudaSuccess) return MLA_ERR_CUDA;
   if (n_merge > 0) {
-    MergeParams mp{reinterpret_cast<const MergeItem*>(scratch + kOffMerge), ap.ws_o, ap.ws_lse, out, lse};
+    MergeParams mp{reinterpret_cast<const MergeItem*>(scratch + kOffMerge),
+                   reinterpret_cast<const int32_t*>(scratch + kOffRefs), ap.ws_o, ap.ws_lse, out, lse};
     if (launch_merge(mp, n_merge, s) != cudaSuccess) return MLA_ERR_CUDA;
   }
   return MLA_OK;

@@ -119,6 +119,12 @@ def test_null_pointers_rejected_by_c_abi():
     assert st == M.MLA_ERR_INVALID_ARGUMENT
     assert lib.mla_plan_check(None) == M.MLA_ERR_INVALID_ARGUMENT
     assert lib.mla_run(None, None, None, None, None, None, None) == M.MLA_ERR_INVALID_ARGUMENT
+    assert lib.mla_plan_update(None, 0, None, None, None, None, None, None) == M.MLA_ERR_INVALID_ARGUMENT
+    assert lib.mla_append_kv(None, None, None, None) == M.MLA_ERR_INVALID_ARGUMENT
+    assert lib.mla_run_append(None, None, None, None, None, None, None, None) == M.MLA_ERR_INVALID_ARGUMENT
+    assert lib.mla_merge_state(None, None, None, None, None, None, 4, None) == M.MLA_ERR_INVALID_ARGUMENT
+    assert lib.mla_merge_state(None, None, None, None, None, None, -1, None) == M.MLA_ERR_INVALID_ARGUMENT
+    assert lib.mla_merge_state(None, None, None, None, None, None, 0, None) == M.MLA_OK  # nothing to do
     lib.mla_plan_destroy(None)  # no-op
 
 

@@ -1,0 +1,306 @@
+"""GPU parity of the entry points around the attention: the latent-cache append, graph
+plans re-planned in place and replayed from a captured CUDA graph, context-only plans
+with the two-state merge, and the shared-prefix cascade.  Every check compares the
+library (through its C ABI) with the fp64 oracle on seeded inputs.
+
+Tolerances as for the attention: bf16 output |err| <= 1e-2 + 1e-2 * |ref|, lse
+|err| <= 1e-3 (and -inf exactly where the oracle has -inf); byte moves are bit-exact.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import paged_head_latent_mla_b200 as M
+from oracle import mla_oracle as O
+from workloads import make_config, make_custom
+
+pytestmark = pytest.mark.gpu
+
+OUT_ATOL, OUT_RTOL, LSE_ATOL = 1e-2, 1e-2, 1e-3
+TIMEOUT_NS = 500_000_000
+DEV = torch.device("cuda:0")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    from paged_head_latent_mla_b200 import _build
+
+    _build.build()
+    return M.load_library()
+
+
+def _plan(d, **kw):
+    return M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=d.num_heads,
+                      page_size=d.page_size, num_pages=d.num_pages, sm_scale=d.sm_scale, causal=d.causal,
+                      wait_timeout_ns=TIMEOUT_NS, **kw)
+
+
+def _check(out, lse, ref_o, ref_l, rows=None):
+    out = out.float().cpu().numpy() if isinstance(out, torch.Tensor) else out
+    lse = lse.cpu().numpy() if isinstance(lse, torch.Tensor) else lse
+    if rows is not None:
+        out, lse, ref_o, ref_l = out[rows], lse[rows], ref_o[rows], ref_l[rows]
+    err = np.abs(out - ref_o)
+    bad = err > OUT_ATOL + OUT_RTOL * np.abs(ref_o)
+    assert not bad.any(), f"out mismatch at {np.argwhere(bad)[:5].tolist()}, max err {err.max():.3e}"
+    inf_r = np.isneginf(ref_l)
+    assert np.array_equal(np.isneginf(lse), inf_r)
+    assert np.abs(lse[~inf_r] - ref_l[~inf_r]).max(initial=0.0) <= LSE_ATOL
+
+
+def _kv_new(T, seed):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn((T, 576), generator=g) * 0.5).to(torch.bfloat16)
+
+
+# ------------------------------------------------------------------------- append
+@pytest.mark.parametrize("H,P", [(128, 64), (16, 16), (64, 128)])
+def test_append_kv_is_bit_exact(H, P):
+    d = make_custom([1, 4, 0, 7, 2], [65, 300, 40, 7, 1000], H, P, seed=61, extra_pool_pages=5)
+    kv_new = _kv_new(int(d.qo_indptr[-1]), 62)
+    plan = _plan(d)
+    cache = d.cache.to(DEV)
+    M.mla_append_kv(plan, kv_new.to(DEV), cache)
+    torch.cuda.synchronize()
+    ref = O.append_latent(d.cache, kv_new, d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, P)
+    got = cache.cpu()
+    assert torch.equal(got, torch.from_numpy(ref).to(torch.bfloat16))  # exact: bf16 values moved as bytes
+    plan.destroy()
+
+
+def test_run_append_attends_the_appended_rows():
+    """mla_run with kv_new: the append runs first (the attention is its programmatic
+    dependent) and the attention sees the new rows, including each token's own."""
+    d = make_custom([1, 3, 1, 6], [200, 129, 4000, 700], 128, 64, seed=63)
+    T = int(d.qo_indptr[-1])
+    kv_new = _kv_new(T, 64)
+    plan = _plan(d)
+    cache = d.cache.to(DEV)
+    out, lse = M.mla_run(plan, d.q_nope.to(DEV), d.q_pe.to(DEV), cache, return_lse=True, kv_new=kv_new.to(DEV))
+    assert M.mla_plan_check(plan) == M.MLA_OK
+    appended = O.append_latent(d.cache, kv_new, d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, 64)
+    assert torch.equal(cache.cpu(), torch.from_numpy(appended).to(torch.bfloat16))
+    ref_o, ref_l = O.mla_attention(d.q_nope, d.q_pe, appended, d.qo_indptr, d.kv_indptr, d.kv_indices,
+                                   d.last_page_len, 64, d.sm_scale, causal=True)
+    _check(out, lse, ref_o, ref_l)
+    plan.destroy()
+
+
+def test_append_rejects_rows_without_slots():
+    d = make_custom([5], [3], 128, 64, seed=65)
+    plan = _plan(d)
+    with pytest.raises(M.MlaError):
+        M.mla_append_kv(plan, _kv_new(5, 1).to(DEV), d.cache.to(DEV))
+    plan.destroy()
+
+
+# ------------------------------------------------------------------------- graph plans
+def _graph_steps():
+    """Steps of one bucket (at most 12 rows, 24 tokens, 1200 page ids) over one pool."""
+    pool = 1400
+    specs = [
+        ([1] * 12, [300 + 211 * i for i in range(12)]),       # decode, no split
+        ([1] * 4, [20000, 16000, 500, 64]),                    # long rows: split + merge
+        ([4, 4, 2], [1500, 900, 3000]),                        # speculative-style
+        ([], []),                                              # an empty step
+        ([1, 1], [1, 40]),                                     # tiny
+        ([7, 1, 1, 1, 1, 1, 1, 1, 1, 1], [2049] + [700] * 9),  # mixed
+    ]
+    return [make_custom(q, k, 128, 64, seed=70 + i, pool_pages=pool) for i, (q, k) in enumerate(specs)]
+
+
+def test_graph_plan_replays_updated_steps():
+    """A CUDA graph captured once around mla_run on a graph plan replays every later step
+    correctly after mla_plan_update re-planned the plan in place."""
+    steps = _graph_steps()
+    TM, H = 24, 128
+    d0 = steps[0]
+    plan = _plan(d0, graph_max_batch=12, graph_max_tokens=TM, graph_max_page_ids=1200)
+    cache = torch.empty((1400, 64, 576), dtype=torch.bfloat16, device=DEV)
+    qn = torch.zeros((TM, H, 512), dtype=torch.bfloat16, device=DEV)
+    qp = torch.zeros((TM, H, 64), dtype=torch.bfloat16, device=DEV)
+    out = torch.empty((TM, H, 512), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((TM, H), dtype=torch.float32, device=DEV)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        M.mla_run(plan, qn, qp, cache, out=out, lse=lse)  # warm-up outside capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        M.mla_run(plan, qn, qp, cache, out=out, lse=lse)
+    for i, d in enumerate(steps):
+        T = int(d.qo_indptr[-1])
+        with torch.cuda.stream(s):
+            reused = M.mla_plan_update(plan, d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len,
+                                       stream=s.cuda_stream)
+            assert reused == (i == 0)
+            cache.copy_(d.cache.to(DEV))
+            if T:
+                qn[:T].copy_(d.q_nope.to(DEV))
+                qp[:T].copy_(d.q_pe.to(DEV))
+            g.replay()
+        torch.cuda.synchronize()
+        assert M.mla_plan_check(plan) == M.MLA_OK
+        if T == 0:
+            continue
+        ref_o, ref_l = O.mla_attention(d.q_nope, d.q_pe, d.cache, d.qo_indptr, d.kv_indptr, d.kv_indices,
+                                       d.last_page_len, 64, d.sm_scale, causal=True)
+        _check(out[:T], lse[:T], ref_o, ref_l)
+        if i == 1:
+            assert M.mla_plan_get_info(plan)["num_merge"] > 0  # the split path replayed too
+    del g
+    plan.destroy()
+
+
+def test_graph_plan_replays_append_and_attention():
+    steps = _graph_steps()[:3]
+    TM, H = 24, 128
+    plan = _plan(steps[0], graph_max_batch=12, graph_max_tokens=TM, graph_max_page_ids=1200)
+    cache = torch.empty((1400, 64, 576), dtype=torch.bfloat16, device=DEV)
+    qn = torch.zeros((TM, H, 512), dtype=torch.bfloat16, device=DEV)
+    qp = torch.zeros((TM, H, 64), dtype=torch.bfloat16, device=DEV)
+    kvn = torch.zeros((TM, 576), dtype=torch.bfloat16, device=DEV)
+    out = torch.empty((TM, H, 512), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((TM, H), dtype=torch.float32, device=DEV)
+    s = torch.cuda.Stream()
+    scratch = torch.empty_like(cache)
+    with torch.cuda.stream(s):
+        M.mla_run(plan, qn, qp, scratch, out=out, lse=lse, kv_new=kvn)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        M.mla_run(plan, qn, qp, cache, out=out, lse=lse, kv_new=kvn)
+    for i, d in enumerate(steps):
+        T = int(d.qo_indptr[-1])
+        kv_new = _kv_new(T, 80 + i)
+        with torch.cuda.stream(s):
+            M.mla_plan_update(plan, d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, stream=s.cuda_stream)
+            cache.copy_(d.cache.to(DEV))
+            qn[:T].copy_(d.q_nope.to(DEV))
+            qp[:T].copy_(d.q_pe.to(DEV))
+            kvn[:T].copy_(kv_new.to(DEV))
+            g.replay()
+        torch.cuda.synchronize()
+        appended = O.append_latent(d.cache, kv_new, d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, 64)
+        assert torch.equal(cache.cpu(), torch.from_numpy(appended).to(torch.bfloat16))
+        ref_o, ref_l = O.mla_attention(d.q_nope, d.q_pe, appended, d.qo_indptr, d.kv_indptr, d.kv_indices,
+                                       d.last_page_len, 64, d.sm_scale, causal=True)
+        _check(out[:T], lse[:T], ref_o, ref_l)
+    del g
+    plan.destroy()
+
+
+def test_plan_update_on_ordinary_plan_grows_and_matches():
+    steps = _graph_steps()
+    plan = _plan(steps[4])
+    for d in (steps[1], steps[5], steps[0]):
+        assert not M.mla_plan_update(plan, d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len)
+        out, lse = M.mla_run(plan, d.q_nope.to(DEV), d.q_pe.to(DEV), d.cache.to(DEV), return_lse=True)
+        assert M.mla_plan_check(plan) == M.MLA_OK
+        ref_o, ref_l = O.mla_attention(d.q_nope, d.q_pe, d.cache, d.qo_indptr, d.kv_indptr, d.kv_indices,
+                                       d.last_page_len, 64, d.sm_scale, causal=True)
+        _check(out, lse, ref_o, ref_l)
+    plan.destroy()
+
+
+# ------------------------------------------------------------------------- context-only + merge
+def _own_token_tables(d):
+    """A second cache holding only each row's own q_b latent rows (copied from the end of
+    its key sequence), with page tables for causal attention among them."""
+    P = d.page_size
+    qo = d.qo_indptr.numpy()
+    k = O.kv_lengths(d.kv_indptr, d.last_page_len, P)
+    pages, kvp, last, rows = [], [0], [], []
+    for b in range(len(qo) - 1):
+        q_b = int(qo[b + 1] - qo[b])
+        keys = O.gather_row_keys(d.cache, d.kv_indptr, d.kv_indices, P, b, int(k[b]))[int(k[b]) - q_b:]
+        n = -(-q_b // P)
+        for p in range(n):
+            blk = np.zeros((P, 576))
+            part = keys[p * P:(p + 1) * P]
+            blk[: len(part)] = part
+            rows.append(blk)
+            pages.append(len(rows) - 1)
+        kvp.append(kvp[-1] + n)
+        last.append(q_b - (n - 1) * P if n else 1)
+    cache2 = torch.from_numpy(np.stack(rows) if rows else np.zeros((1, P, 576))).to(torch.bfloat16)
+    return cache2, torch.tensor(kvp, dtype=torch.int32), torch.tensor(pages, dtype=torch.int32), \
+        torch.tensor(last, dtype=torch.int32)
+
+
+def test_context_only_merged_with_own_tokens_equals_full_attention():
+    d = make_custom([3, 1, 9, 2], [3 + 500, 1 + 64, 9 + 0, 2 + 2000], 128, 64, seed=91)
+    ctx = _plan(d, context_only=True)
+    qn, qp = d.q_nope.to(DEV), d.q_pe.to(DEV)
+    out_c, lse_c = M.mla_run(ctx, qn, qp, d.cache.to(DEV), return_lse=True)
+    assert M.mla_plan_check(ctx) == M.MLA_OK
+    ref_c = O.mla_attention(d.q_nope, d.q_pe, d.cache, d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len,
+                            64, d.sm_scale, context_only=True)
+    _check(out_c, lse_c, *ref_c)
+    assert list(M.mla_plan_describe(ctx)["kv_len"]) == [500, 64, 0, 2000]
+    cache2, kvp2, idx2, last2 = _own_token_tables(d)
+    own = M.mla_plan(d.qo_indptr, kvp2, idx2, last2, num_heads=128, page_size=64, num_pages=cache2.shape[0],
+                     sm_scale=d.sm_scale, causal=True)
+    out_s, lse_s = M.mla_run(own, qn, qp, cache2.to(DEV), return_lse=True)
+    out, lse = M.mla_merge_state(out_c, lse_c, out_s, lse_s)
+    ref_o, ref_l = O.mla_attention(d.q_nope, d.q_pe, d.cache, d.qo_indptr, d.kv_indptr, d.kv_indices,
+                                   d.last_page_len, 64, d.sm_scale, causal=True)
+    _check(out, lse, ref_o, ref_l)
+    ctx.destroy()
+    own.destroy()
+
+
+def test_merge_state_matches_oracle_including_empty_states():
+    g = torch.Generator().manual_seed(93)
+    R = 1000
+    oa = (torch.randn((R, 512), generator=g)).to(torch.bfloat16)
+    ob = (torch.randn((R, 512), generator=g)).to(torch.bfloat16)
+    la = torch.randn(R, generator=g) * 4
+    lb = torch.randn(R, generator=g) * 4
+    la[::7] = -float("inf")
+    lb[::11] = -float("inf")
+    la[5], lb[5] = 80.0, -80.0  # one state dominates completely
+    out, lse = M.mla_merge_state(oa.to(DEV), la.to(DEV), ob.to(DEV), lb.to(DEV))
+    ref_o, ref_l = O.merge_states(oa, la, ob, lb)
+    _check(out, lse, ref_o, ref_l)
+    both = (np.arange(R) % 77) == 0
+    assert np.all(out.float().cpu().numpy()[both] == 0)
+    # in place: out aliases out_a
+    a2 = oa.to(DEV)
+    M.mla_merge_state(a2, la.to(DEV), ob.to(DEV), lb.to(DEV), out=a2)
+    assert torch.equal(a2.cpu(), out.cpu())
+
+
+# ------------------------------------------------------------------------- cascade
+@pytest.mark.parametrize("H,P,q", [(128, 64, 4), (16, 16, 4), (16, 16, 3), (64, 32, 1)])
+def test_cascade_matches_oracle(H, P, q):
+    B, group = 8, 4
+    k = [1024 + q + 37 * i for i in range(B)]
+    d = make_custom([q] * B, k, H, P, shared_group=group, shared_pages=1024 // P, seed=95 + H + q)
+    plan = _plan(d, cascade=True)
+    assert M.mla_plan_get_info(plan)["num_cascade"] > 0
+    out, lse = M.mla_run(plan, d.q_nope.to(DEV), d.q_pe.to(DEV), d.cache.to(DEV), return_lse=True)
+    assert M.mla_plan_check(plan) == M.MLA_OK
+    ref_o, ref_l = O.mla_attention(d.q_nope, d.q_pe, d.cache, d.qo_indptr, d.kv_indptr, d.kv_indices,
+                                   d.last_page_len, P, d.sm_scale, causal=True)
+    _check(out, lse, ref_o, ref_l)
+    plan.destroy()
+
+
+@pytest.mark.slow
+def test_cascade_full_size_speculative_sampled():
+    """The speculative shared-prefix workload (128 rows, 4 queries each, groups of 8
+    sharing 1024 keys) with the cascade on, checked on sampled tokens."""
+    d = make_config("spec_shared_prefix")
+    plan = _plan(d, cascade=True)
+    info = M.mla_plan_get_info(plan)
+    assert info["num_cascade"] >= 16 * 32
+    out, lse = M.mla_run(plan, d.q_nope.to(DEV), d.q_pe.to(DEV), d.cache.to(DEV), return_lse=True)
+    assert M.mla_plan_check(plan) == M.MLA_OK
+    qo = d.qo_indptr.numpy()
+    toks = sorted({int(qo[b]) for b in (0, 7, 8, 63, 127)} | {int(qo[b + 1] - 1) for b in (0, 9, 127)})
+    ref_o, ref_l = O.mla_attention(d.q_nope, d.q_pe, d.cache, d.qo_indptr, d.kv_indptr, d.kv_indices,
+                                   d.last_page_len, d.page_size, d.sm_scale, causal=True, tokens=toks)
+    _check(out, lse, ref_o, ref_l, rows=np.asarray(toks))
+    plan.destroy()

@@ -9,7 +9,11 @@
 * closed forms (zero query, equal keys, a single visible key);
 * invariances (physical page permutation; causal == non-causal for one query);
 * the LSE merge identity (flashinfer_mla page, FlashInferMLAManager.run: the lse
-  exists to merge key segments), with brute-force splits.
+  exists to merge key segments), with brute-force splits;
+* the cache append against a walk over the page lists and a hand-derived example,
+  and its round trip through the paged gather;
+* context-only attention merged with attention over the step's own tokens equals
+  full causal attention (the two key sets partition every query's visible keys).
 
 The ``check_*`` functions take the oracle module as an argument so that the
 mutation tests at the bottom can plant plausible mistakes in a copy of the
@@ -262,6 +266,87 @@ def check_kv_lengths(oracle):
                 j += 1
 
 
+def _walk_slots(kv_indptr, kv_indices, last, P, b):
+    """The row's (page, slot) pairs in logical key order, by walking its page list."""
+    out = []
+    n = kv_indptr[b + 1] - kv_indptr[b]
+    for p in range(n):
+        for s_ in range(last[b] if p == n - 1 else P):
+            out.append((int(kv_indices[kv_indptr[b] + p]), s_))
+    return out
+
+
+def check_append_slots(oracle):
+    # hand-derived example
+    with open(os.path.join(GOLDEN, "append_tiny.json")) as f:
+        g = json.load(f)
+    P = g["page_size"]
+    cache = np.zeros((g["num_pages"], P, D_C + D_R))
+    T = g["qo_indptr"][-1]
+    new = np.arange(T, dtype=np.float64)[:, None] + 1.0 + np.zeros((T, D_C + D_R))
+    out = oracle.append_latent(cache, new, g["qo_indptr"], g["kv_indptr"], g["kv_indices"], g["last_page_len"], P)
+    for t, (page, slot) in enumerate(g["expected_page_slot"]):
+        assert np.all(out[page, slot] == t + 1.0)
+    assert np.count_nonzero(out.any(axis=-1)) == T  # nothing else written
+    # random tables: the last q_b slots of each row's walk receive the new rows in
+    # order, every other slot is unchanged, and the paged gather reads them back
+    d = _paged([3, 0, 5, 1], [40, 7, 70, 1], 2, 16, seed=11)
+    new = np.random.default_rng(12).normal(size=(9, D_C + D_R))
+    out = oracle.append_latent(d["cache"], new, d["qo_indptr"], d["kv_indptr"], d["kv_indices"],
+                               d["last_page_len"], 16)
+    touched = np.zeros(d["cache"].shape[:2], dtype=bool)
+    qo = d["qo_indptr"]
+    for b in range(4):
+        slots = _walk_slots(d["kv_indptr"], d["kv_indices"], d["last_page_len"], 16, b)
+        q_b = qo[b + 1] - qo[b]
+        for i, (page, slot) in enumerate(slots[len(slots) - q_b:]):
+            assert np.array_equal(out[page, slot], new[qo[b] + i])
+            touched[page, slot] = True
+        k_b = len(slots)
+        keys = oracle.gather_row_keys(out, d["kv_indptr"], d["kv_indices"], 16, b, k_b)
+        assert np.array_equal(keys[k_b - q_b:], new[qo[b]:qo[b + 1]])
+    assert np.array_equal(out[~touched], d["cache"][~touched])
+    with pytest.raises(ValueError):
+        oracle.append_latent(d["cache"], new[:6], [0, 6], [0, 1], [0], [5], 16)
+
+
+def check_context_only_merge(oracle):
+    """Context-only attention (keys j < k_b - q_b) merged by LSE with attention over the
+    row's own q_b tokens (causal among themselves) equals full causal attention."""
+    P, H = 16, 3
+    q_lens, k_lens = [4, 1, 7, 2], [4 + 37, 1 + 16, 7 + 0, 2 + 50]
+    d = _paged(q_lens, k_lens, H, P, seed=21)
+    full_o, full_l = oracle.mla_attention(d["q_nope"], d["q_pe"], d["cache"], d["qo_indptr"], d["kv_indptr"],
+                                          d["kv_indices"], d["last_page_len"], P, SCALE, causal=True)
+    ctx_o, ctx_l = oracle.mla_attention(d["q_nope"], d["q_pe"], d["cache"], d["qo_indptr"], d["kv_indptr"],
+                                        d["kv_indices"], d["last_page_len"], P, SCALE, causal=True,
+                                        context_only=True)
+    # own-token attention written out directly: query i sees own tokens 0..i
+    qo = d["qo_indptr"]
+    own_o = np.zeros_like(full_o)
+    own_l = np.full(full_l.shape, -np.inf)
+    for b in range(4):
+        slots = _walk_slots(d["kv_indptr"], d["kv_indices"], d["last_page_len"], P, b)
+        q_b = qo[b + 1] - qo[b]
+        own = np.stack([d["cache"][pg, sl] for pg, sl in slots[len(slots) - q_b:]])  # [q_b, 576]
+        for i in range(q_b):
+            t = qo[b] + i
+            q = np.concatenate([d["q_nope"][t], d["q_pe"][t]], axis=-1)
+            s_ = (q @ own[: i + 1].T) * SCALE
+            m = s_.max(axis=1, keepdims=True)
+            e = np.exp(s_ - m)
+            own_l[t] = (m + np.log(e.sum(axis=1, keepdims=True)))[:, 0]
+            own_o[t] = (e / e.sum(axis=1, keepdims=True)) @ own[: i + 1, :D_C]
+    mo, ml = oracle.merge_states(ctx_o, ctx_l, own_o, own_l)
+    assert np.allclose(mo, full_o, rtol=0, atol=1e-12) and np.allclose(ml, full_l, rtol=0, atol=1e-12)
+    # a row with no stored context attends nothing in context-only mode
+    t = qo[2]
+    assert np.all(ctx_o[t] == 0) and np.all(ctx_l[t] == -np.inf)
+    with pytest.raises(ValueError):
+        oracle.mla_attention(d["q_nope"][:3], d["q_pe"][:3], d["cache"], [0, 3], [0, 1], d["kv_indices"][:1],
+                             [2], P, SCALE, context_only=True)
+
+
 ALL_CHECKS = [
     check_absorbed_equals_explicit,
     check_against_sdpa,
@@ -273,6 +358,8 @@ ALL_CHECKS = [
     check_lse_merge,
     check_empty_and_overhang,
     check_kv_lengths,
+    check_append_slots,
+    check_context_only_merge,
 ]
 
 
@@ -367,8 +454,34 @@ def _mut_merge_sign(mod):
     mod.merge_states = f
 
 
+def _mut_append_start_aligned(mod):
+    # wrong: the step's tokens written at the start of the row instead of its end
+    def f(cache, kv_new, qo_indptr, kv_indptr, kv_indices, last_page_len, page_size):
+        out = mod._f64(cache).copy()
+        new = mod._f64(kv_new)
+        qo = mod._i64(qo_indptr)
+        for b in range(len(qo) - 1):
+            for i in range(int(qo[b + 1] - qo[b])):
+                page, slot = mod.key_location(kv_indptr, kv_indices, page_size, b, i)
+                out[page, slot] = new[qo[b] + i]
+        return out
+
+    mod.append_latent = f
+
+
+def _mut_context_includes_own(mod):
+    # wrong: a context-only query also sees the step's own tokens
+    orig = mod.mla_attention
+
+    def f(*a, context_only=False, **kw):
+        return orig(*a, context_only=False, **{**kw, "causal": False}) if context_only else orig(*a, **kw)
+
+    mod.mla_attention = f
+
+
 MUTATIONS = [_mut_start_aligned, _mut_drop_rope, _mut_wrong_scale, _mut_log2_lse, _mut_value_includes_rope,
-             _mut_kv_len_off_by_one, _mut_slot_transposed, _mut_merge_sign]
+             _mut_kv_len_off_by_one, _mut_slot_transposed, _mut_merge_sign, _mut_append_start_aligned,
+             _mut_context_includes_own]
 
 
 @pytest.mark.parametrize("mutate", MUTATIONS, ids=lambda m: m.__name__)

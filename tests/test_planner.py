@@ -17,48 +17,78 @@ def plan_tables(d, **kw):
                       host_only=True, **kw)
 
 
-def check_layout(d, desc, num_sms=148):
+def check_layout(d, desc, context_only=False):
+    """Check a plan's work items, merge records and merge references against the
+    oracle's reading of the tables: every visible key of every query is covered exactly
+    once; an item's visibility rule reproduces the oracle's; partial results occupy
+    disjoint workspace rows; and every token whose items are partials is combined by
+    exactly one merge record that references each of them exactly once."""
     H, P = d.num_heads, d.page_size
     qo = d.qo_indptr.numpy().astype(np.int64)
     kvp = d.kv_indptr.numpy().astype(np.int64)
+    idx = d.kv_indices.numpy()
     B = len(qo) - 1
-    k_oracle = O.kv_lengths(kvp, d.last_page_len.numpy(), P)
-    assert np.array_equal(desc["kv_len"].astype(np.int64), k_oracle)
+    k_full = O.kv_lengths(kvp, d.last_page_len.numpy(), P)
+    q_len = np.diff(qo)
+    k_att = k_full - q_len if context_only else k_full  # keys the queries attend
+    assert np.array_equal(desc["kv_len"].astype(np.int64), k_att)
+    causal = d.causal and not context_only
 
-    work, merge = desc["work"], desc["merge"]
+    def vis_of(b, i):
+        return O.visible_keys(int(k_att[b]), int(q_len[b]), int(i), causal)
+
+    work, merge, refs = desc["work"], desc["merge"], desc["refs"]
     info = desc["info"]
     assert info["num_work"] == len(work) and info["num_merge"] == len(merge)
-    # token -> batch row
+    assert info["num_merge_refs"] == len(refs)
+    T = int(qo[-1])
     row_of_token = np.repeat(np.arange(B), np.diff(qo))
-    # coverage[t] = list of (key_begin, key_end) from items covering token t
-    cover = [[] for _ in range(int(qo[-1]))]
-    partial_seen = []
-    for (q_row0, n_rows, page_base, kv_len, kb, ke, diag, partial) in work:
+    cover = [[] for _ in range(T)]  # (key_begin, key_end, item index)
+    ws_used = []
+    n_cascade = 0
+    for wi, (q_row0, n_rows, page_base, kv_len, kb, ke, diag, partial) in enumerate(work):
         assert q_row0 % H == 0 and n_rows % H == 0 and 0 < n_rows <= 128
-        t0 = q_row0 // H
-        ntok = n_rows // H
-        b = row_of_token[t0]
-        assert row_of_token[t0 + ntok - 1] == b, "a tile crosses batch rows"
-        assert page_base == kvp[b]  # so key j -> kv_indices[page_base + j // P], slot j % P
-        assert kv_len == k_oracle[b]
-        assert kb % M.MLA_KEY_TILE == 0 and kb <= ke or (kb == 0 and ke == 0)
-        q_b = qo[b + 1] - qo[b]
-        i0 = t0 - qo[b]
-        vis_hi = O.visible_keys(int(k_oracle[b]), int(q_b), int(i0 + ntok - 1), d.causal)
-        assert ke <= vis_hi
-        for tt in range(ntok):
-            i = i0 + tt
-            vis = O.visible_keys(int(k_oracle[b]), int(q_b), int(i), d.causal)
-            # the kernel's rule: keys < clamp(diag + tt + 1, 0, kv_len)
-            assert min(max(diag + tt + 1, 0), kv_len) == vis
-            cover[t0 + tt].append((kb, ke))
+        t0, ntok = q_row0 // H, n_rows // H
+        rows = set(row_of_token[t0:t0 + ntok].tolist())
+        assert kb % M.MLA_KEY_TILE == 0 and (kb <= ke or (kb == ke))
+        if len(rows) > 1 or (kv_len != k_att[row_of_token[t0]]):
+            # a cascade item: a shared prefix [0, kv_len) seen in full by every row
+            n_cascade += 1
+            assert partial >= 0 and kb >= 0 and ke <= kv_len and diag >= kv_len
+            # it reads some row's pages (the group's first); every row it serves names
+            # the same page ids for those keys
+            assert page_base in set(kvp[:-1].tolist())
+            npg = -(-int(kv_len) // P)
+            for b in rows:
+                assert np.array_equal(idx[kvp[b]:kvp[b] + npg], idx[page_base:page_base + npg])
+            for tt in range(ntok):
+                b = row_of_token[t0 + tt]
+                assert kv_len <= vis_of(b, t0 + tt - qo[b])
+                assert min(max(diag + tt + 1, 0), kv_len) == kv_len
+                cover[t0 + tt].append((kb, ke, wi))
+        else:
+            b = row_of_token[t0]
+            assert page_base == kvp[b]  # so key j -> kv_indices[page_base + j // P], slot j % P
+            i0 = t0 - qo[b]
+            assert ke <= max(vis_of(b, i0 + ntok - 1), kb)
+            for tt in range(ntok):
+                # the kernel's rule: keys < clamp(diag + tt + 1, 0, kv_len)
+                assert min(max(diag + tt + 1, 0), kv_len) == vis_of(b, i0 + tt)
+                cover[t0 + tt].append((kb, ke, wi))
         if partial >= 0:
-            partial_seen.append(partial)
+            ws_used.append((int(partial), int(partial) + int(n_rows)))
+    # (a single-row prefix item whose prefix is all of the row reads like an ordinary one)
+    assert n_cascade <= info["num_cascade"]
+    # partial results occupy disjoint workspace rows
+    ws_used.sort()
+    for (a0, a1), (b0, b1) in zip(ws_used, ws_used[1:]):
+        assert a1 <= b0
+    assert info["num_partials"] == len(ws_used)
     # every visible key of every query is covered exactly once
-    for t in range(int(qo[-1])):
+    for t in range(T):
         b = row_of_token[t]
-        vis = O.visible_keys(int(k_oracle[b]), int(qo[b + 1] - qo[b]), int(t - qo[b]), d.causal)
-        spans = sorted(cover[t])
+        vis = vis_of(b, t - qo[b])
+        spans = sorted((kb, ke) for kb, ke, _ in cover[t])
         assert spans, f"token {t} uncovered"
         pos = 0
         for (kb, ke) in spans:
@@ -66,18 +96,27 @@ def check_layout(d, desc, num_sms=148):
                 continue
             assert kb == pos, f"token {t}: gap/overlap at {pos} vs {kb}"
             pos = ke
-        assert pos >= vis and pos <= max(vis, spans[-1][1])
-        # no key beyond the tile's vis_hi is ever used, and keys beyond vis are masked
-    # partial slots: each used exactly once, grouped contiguously per merge record
-    assert sorted(partial_seen) == list(range(info["num_partials"]))
-    for (q_row0, n_rows, first, n) in merge:
-        assert n >= 2
-        items = [w for w in work if w[7] >= first and w[7] < first + n]
-        assert len(items) == n
-        assert all(w[0] == q_row0 and w[1] == n_rows for w in items)
-        spans = sorted((w[4], w[5]) for w in items)
-        for a, b2 in zip(spans, spans[1:]):
-            assert a[1] == b2[0] and a[1] % M.MLA_KEY_TILE == 0
+        assert pos >= vis  # keys past a token's own limit are masked by the kernel's rule
+    # merges: a token with partial items is combined once, from exactly those partials
+    merged_by = [None] * T
+    for mi, (q_row0, n_rows, first, n) in enumerate(merge):
+        assert n >= 1 and q_row0 % H == 0 and n_rows % H == 0
+        for t in range(q_row0 // H, (q_row0 + n_rows) // H):
+            assert merged_by[t] is None
+            merged_by[t] = mi
+        assert 0 <= first and first + n <= len(refs)
+    for t in range(T):
+        parts = [wi for _, _, wi in cover[t] if work[wi][7] >= 0]
+        finals = [wi for _, _, wi in cover[t] if work[wi][7] < 0]
+        if not parts:
+            assert merged_by[t] is None and len(finals) == 1
+            continue
+        assert not finals and merged_by[t] is not None
+        q_row0, n_rows, first, n = merge[merged_by[t]]
+        # the workspace row that holds token t's head 0 in each referenced partial
+        want = sorted(int(work[wi][7]) + (t * H - int(work[wi][0])) for wi in parts)
+        got = sorted(int(r) + (t * H - int(q_row0)) for r in refs[first:first + n])
+        assert got == want
     return True
 
 
@@ -143,3 +182,94 @@ def test_no_split_for_small_decode():
     d = make_config("tiny_decode", tables_only=True)
     desc = M.mla_plan_describe(plan_tables(d))
     assert desc["info"]["num_merge"] == 0 and desc["info"]["num_work"] == 2
+
+
+@pytest.mark.parametrize("H,P,q", [(128, 64, 4), (16, 16, 4), (16, 16, 3), (32, 32, 1), (64, 128, 2)])
+def test_cascade_layout_covers_once_and_groups_rows(H, P, q):
+    """Shared-prefix cascade (consecutive rows naming the same first pages attend them
+    together): coverage, visibility and merge references stay exact, and every group
+    with a long enough shared prefix gets prefix items spanning its rows' queries."""
+    B, group, shared = 12, 4, (1024 // P)
+    k = [1024 + q + 13 * i for i in range(B)]
+    d = make_custom([q] * B, k, H, P, shared_group=group, shared_pages=shared, tables_only=True, seed=H + P)
+    p = plan_tables(d, cascade=True)
+    desc = M.mla_plan_describe(p)
+    check_layout(d, desc)
+    info = desc["info"]
+    # shared prefix keys = 1024 (a multiple of 64, visible in full to every query)
+    rows_per_item = min(128, max(H * q, (128 // (H * q)) * H * q))
+    expect_items = (B // group) * (-(-group * q * H // rows_per_item))
+    assert info["num_cascade"] >= expect_items
+    prefix = [w for w in desc["work"] if w[3] == 1024 and w[6] >= 1024]
+    assert len(prefix) >= expect_items
+    # without the option, nothing is cascaded
+    assert M.mla_plan_describe(plan_tables(d))["info"]["num_cascade"] == 0
+
+
+def test_cascade_skips_groups_without_a_full_tile_of_prefix():
+    d = make_custom([2] * 8, [700] * 8, 128, 16, shared_group=4, shared_pages=3, tables_only=True)
+    desc = M.mla_plan_describe(plan_tables(d, cascade=True))
+    check_layout(d, desc)
+    assert desc["info"]["num_cascade"] == 0  # 48 shared keys < one 64-key tile
+
+
+@pytest.mark.parametrize("split", [0, -1, 128])
+def test_context_only_layout(split):
+    """Context-only plans attend keys [0, k_b - q_b) of every row with no causal mask."""
+    rng = np.random.default_rng(7 + split)
+    q = rng.integers(1, 40, 10).tolist()
+    k = [qi + int(c) for qi, c in zip(q, rng.integers(0, 900, 10))]
+    k[2] = q[2]  # no stored context
+    d = make_custom(q, k, 64, 32, tables_only=True, seed=3)
+    desc = M.mla_plan_describe(plan_tables(d, context_only=True, split_keys=split))
+    check_layout(d, desc, context_only=True)
+    # a row whose tables lack slots for its own tokens is rejected
+    bad = make_custom([5], [3], 64, 32, tables_only=True)
+    with pytest.raises(M.MlaError):
+        plan_tables(bad, context_only=True)
+
+
+def test_update_recognises_an_unchanged_step_and_replans_otherwise():
+    # one page pool for both steps: a plan's geometry (num_pages) is fixed
+    d1 = make_custom([1] * 6, [300, 900, 64, 4000, 17, 2000], 128, 64, tables_only=True, seed=1, pool_pages=400)
+    d2 = make_custom([2] * 5, [700, 60, 3000, 128, 9000], 128, 64, tables_only=True, seed=2, pool_pages=400)
+    p = plan_tables(d1)
+    assert M.mla_plan_update(p, d1.qo_indptr, d1.kv_indptr, d1.kv_indices, d1.last_page_len)
+    assert not M.mla_plan_update(p, d2.qo_indptr, d2.kv_indptr, d2.kv_indices, d2.last_page_len)
+    check_layout(d2, M.mla_plan_describe(p))
+    assert M.mla_plan_update(p, d2.qo_indptr, d2.kv_indptr, d2.kv_indices, d2.last_page_len)
+    # one changed page id is a different step
+    kvi = d2.kv_indices.clone()
+    kvi[3] = (int(kvi[3]) + 1) % d2.num_pages
+    assert not M.mla_plan_update(p, d2.qo_indptr, d2.kv_indptr, kvi, d2.last_page_len)
+
+
+def test_graph_plan_bounds_hold_across_steps():
+    """A graph plan's layout fits its bucket's fixed capacity for every step that fits
+    the bucket; a step beyond the bucket is rejected and leaves the plan as it was."""
+    kw = dict(graph_max_batch=16, graph_max_tokens=64, graph_max_page_ids=2048)
+    d0 = make_custom([1] * 16, [100 + 300 * i for i in range(16)], 128, 64, tables_only=True, seed=4,
+                     pool_pages=4096)
+    p = plan_tables(d0, **kw)
+    cap = M.mla_plan_get_info(p)["work_capacity"]
+    assert M.mla_plan_get_info(p)["graph"] == 1
+    rng = np.random.default_rng(5)
+    for step in range(6):
+        B = int(rng.integers(1, 17))
+        q = rng.integers(1, 5, B).tolist()
+        k = [int(qi + x) for qi, x in zip(q, rng.integers(0, 8000, B))]
+        d = make_custom(q, k, 128, 64, tables_only=True, seed=10 + step, pool_pages=4096)
+        if int(d.kv_indptr[-1]) > 2048 or sum(q) > 64:
+            continue
+        M.mla_plan_update(p, d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len)
+        desc = M.mla_plan_describe(p)
+        check_layout(d, desc)
+        assert desc["info"]["num_work"] <= cap and desc["info"]["work_capacity"] == cap
+    too_many = make_custom([1] * 17, [64] * 17, 128, 64, tables_only=True, pool_pages=4096)
+    before = M.mla_plan_describe(p)["work"].copy()
+    with pytest.raises(M.MlaError):
+        M.mla_plan_update(p, too_many.qo_indptr, too_many.kv_indptr, too_many.kv_indices, too_many.last_page_len)
+    assert np.array_equal(M.mla_plan_describe(p)["work"], before)
+    # the three bounds go together
+    with pytest.raises(M.MlaError):
+        plan_tables(d0, graph_max_batch=16, graph_max_tokens=64)
