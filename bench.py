@@ -49,6 +49,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle CPU-baseline budget (0: skip)")
     ap.add_argument("--soak", type=float, default=1.5, help="untimed seconds of steps while clocks are sampled")
     ap.add_argument("--copies", type=int, default=0, help="HBM copies of the inputs to rotate (0: auto)")
+    ap.add_argument("--no-next", action="store_true",
+                    help="skip the measurements of graph replay, append, cascade and plan reuse")
     return ap.parse_args()
 
 
@@ -225,7 +227,7 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------------------- native leg
-def make_runner(d, device, n_copies, timing=True):
+def make_runner(d, device, n_copies, timing=True, plan_kw=None):
     """Plan once; keep `n_copies` copies of the inputs in HBM and rotate through them so
     consecutive steps never find their inputs in L2.  With `timing` the plan records CUDA
     events around each of its launches (kernel durations for the roofline); those events
@@ -238,7 +240,7 @@ def make_runner(d, device, n_copies, timing=True):
 
     plan = M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=d.num_heads,
                       page_size=d.page_size, num_pages=d.num_pages, sm_scale=d.sm_scale, causal=d.causal,
-                      debug_flags=M.MLA_DEBUG_KERNEL_TIMING if timing else 0)
+                      debug_flags=M.MLA_DEBUG_KERNEL_TIMING if timing else 0, **(plan_kw or {}))
     copies = []
     for _ in range(n_copies):
         copies.append((d.q_nope.to(device), d.q_pe.to(device), d.cache.to(device)))
@@ -266,7 +268,7 @@ def input_bytes(d):
     return d.cache.numel() * 2 + d.q_nope.numel() * 2 + d.q_pe.numel() * 2
 
 
-def time_workload(d, device, steps, warmup, dist=None, soak_s=0.0, sampler=None, copies=0):
+def time_workload(d, device, steps, warmup, dist=None, soak_s=0.0, sampler=None, copies=0, plan_kw=None):
     """Two timed regions over the same resident inputs: K steps through a plain plan (the
     product path: the step value), then K steps through a plan that records events
     around each launch (the per-kernel durations for the roofline)."""
@@ -278,10 +280,10 @@ def time_workload(d, device, steps, warmup, dist=None, soak_s=0.0, sampler=None,
     free, _ = torch.cuda.mem_get_info(device)
     while n_copies > 1 and n_copies * input_bytes(d) > 0.6 * free:
         n_copies -= 1
-    plan, step, out, lse, copies = make_runner(d, device, n_copies, timing=False)
+    plan, step, out, lse, copies = make_runner(d, device, n_copies, timing=False, plan_kw=plan_kw)
     tplan = M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=d.num_heads,
                        page_size=d.page_size, num_pages=d.num_pages, sm_scale=d.sm_scale, causal=d.causal,
-                       debug_flags=M.MLA_DEBUG_KERNEL_TIMING)
+                       debug_flags=M.MLA_DEBUG_KERNEL_TIMING, **(plan_kw or {}))
     lib = M.load_library()
     import ctypes
     stream = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
@@ -380,7 +382,9 @@ def time_e2e(d, device, steps, warmup):
         st = M.mla_plan_check(plan)  # synchronises and reads the 4-byte status word
         if st != 0:
             raise M.MlaError(st, "e2e")
-        plan_bytes = 256 + 32 * info["num_work"] + 16 * info["num_merge"] + 4 * int(d.kv_indptr[-1])
+        # work list, merge list and references, append rows, page table
+        plan_bytes = (32 * info["num_work"] + 16 * info["num_merge"] + 4 * info["num_merge_refs"] + 4 * T +
+                      4 * int(d.kv_indptr[-1]))
         h2d[0] = plan_bytes + qn_h.numel() * 2 + qp_h.numel() * 2
         plan.destroy()
 
@@ -420,6 +424,161 @@ def summarise(d, res, peaks):
         "kv_bytes": w["kv_bytes"],
         "flops": w["flops"],
     }
+
+
+def _events_ms(fn, device, n, flush=None):
+    """Mean device time of `fn` over n calls, each bracketed by its own CUDA events on the
+    current stream; `flush` (outside the events) runs before every call."""
+    import torch
+
+    ms = 0.0
+    for _ in range(n):
+        if flush is not None:
+            flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize(device)
+        ms += a.elapsed_time(b)
+    return ms / n
+
+
+def measure_next_rows(device, peaks):
+    """The entry points around the attention, each on its own workload:
+    * graph replay: the tiny decode step replayed from a captured CUDA graph (a graph
+      plan) against the same step launched eagerly, device time per step (L2-warm: the
+      step reads 215 KB, so this is launch latency);
+    * append: mla_append_kv of the mixed chunked-prefill step's 4156 tokens (1152 B read
+      and written per token), L2 flushed before each launch, against HBM bandwidth;
+    * cascade: the speculative shared-prefix rows at 16 heads with and without the cascade;
+    * plan reuse: host time of mla_plan_update on an unchanged decode step (skipped
+      re-plan) against a changed one and a fresh mla_plan."""
+    import torch
+
+    import paged_head_latent_mla_b200 as M
+    from workloads import make_config, make_custom
+
+    res = {}
+    stream = torch.cuda.current_stream(device)
+
+    # --- graph replay vs eager, tiny decode
+    d = make_config("tiny_decode")
+    qn, qp, cache = d.q_nope.to(device), d.q_pe.to(device), d.cache.to(device)
+    T, H = d.total_tokens, d.num_heads
+    out = torch.empty((T, H, 512), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((T, H), dtype=torch.float32, device=device)
+    eager = M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=H,
+                       page_size=d.page_size, num_pages=d.num_pages, sm_scale=d.sm_scale, causal=d.causal)
+    gplan = M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=H,
+                       page_size=d.page_size, num_pages=d.num_pages, sm_scale=d.sm_scale, causal=d.causal,
+                       graph_max_batch=d.batch, graph_max_tokens=T, graph_max_page_ids=int(d.kv_indptr[-1]))
+    n = 200
+    for _ in range(5):
+        M.mla_run(eager, qn, qp, cache, out=out, lse=lse)
+        M.mla_run(gplan, qn, qp, cache, out=out, lse=lse)
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(n):
+        M.mla_run(eager, qn, qp, cache, out=out, lse=lse)
+    b.record()
+    torch.cuda.synchronize(device)
+    eager_us = a.elapsed_time(b) / n * 1e3
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(device)
+    s.wait_stream(stream)
+    with torch.cuda.graph(g, stream=s):
+        for _ in range(10):
+            M.mla_run(gplan, qn, qp, cache, out=out, lse=lse)
+    torch.cuda.synchronize(device)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize(device)
+    a.record()
+    for _ in range(n // 10):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize(device)
+    graph_us = a.elapsed_time(b) / n * 1e3
+    for pl in (eager, gplan):
+        if M.mla_plan_check(pl) != 0:
+            raise M.MlaError(M.mla_plan_check(pl), "graph replay")
+    res["graph_replay_tiny_decode"] = {
+        "eager_us_per_step": eager_us, "graph_us_per_step": graph_us,
+        "work_capacity": M.mla_plan_get_info(gplan)["work_capacity"],
+        "note": "10 steps per captured graph; both on the same inputs, L2-warm (215 KB per step)"}
+    del g
+    eager.destroy()
+    gplan.destroy()
+
+    # --- append bandwidth, mixed chunked-prefill tokens
+    d = make_config("mixed_prefill")
+    T = d.total_tokens
+    cache = d.cache.to(device)
+    kv_new = (torch.randn((T, 576), generator=torch.Generator().manual_seed(5)) * 0.5).to(torch.bfloat16).to(device)
+    plan = M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=d.num_heads,
+                      page_size=d.page_size, num_pages=d.num_pages, sm_scale=d.sm_scale, causal=d.causal)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    for _ in range(3):
+        M.mla_append_kv(plan, kv_new, cache)
+    ms = _events_ms(lambda: M.mla_append_kv(plan, kv_new, cache), device, 20, flush=lambda: flush.fill_(1.0))
+    moved = 2 * 1152 * T
+    res["append_mixed_prefill"] = {"tokens": T, "us": ms * 1e3, "bytes": moved, "gbs": moved / (ms * 1e-3) / 1e9,
+                                   "frac_hbm": moved / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                   "note": "L2 flushed before each launch; 1152 B read + 1152 B written per token"}
+    plan.destroy()
+    del cache, flush, kv_new
+    torch.cuda.empty_cache()
+
+    # --- cascade on/off: the speculative shared-prefix rows with 16 query heads (with 128
+    # heads a token fills a query tile by itself and the planner applies no cascade)
+    t = make_config("spec_shared_prefix", tables_only=True)
+    d = make_custom(t.q_lens, t.kv_lens, 16, 64, shared_group=8, shared_pages=16, seed=0,
+                    name="spec_shared_prefix_h16")
+    base = summarise(d, time_workload(d, device, 20, 3), peaks)
+    casc_res = time_workload(d, device, 20, 3, plan_kw={"cascade": True})
+    casc = summarise(d, casc_res, peaks)
+    res["cascade_spec_shared_prefix_h16"] = {
+        "off_tflops": base["tflops"], "on_tflops": casc["tflops"],
+        "off_us": base["us_per_step"], "on_us": casc["us_per_step"],
+        "off_kv_gbs": base["kv_gbs"], "on_kv_gbs": casc["kv_gbs"],
+        "cascade_items": casc_res["info"]["num_cascade"], "work_items": casc_res["info"]["num_work"],
+        "note": "rows, lengths and prefix groups of spec_shared_prefix with H=16: a prefix tile packs two rows' "
+                "4 x 16 query rows; TFLOP/s and GB/s count the same algorithmic work either way"}
+    del d
+    torch.cuda.empty_cache()
+
+    # --- plan reuse, host time
+    d = make_config("decode_b64", tables_only=True)
+    d2 = make_config("decode_b64", seed=1, tables_only=True)
+    plan = M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=d.num_heads,
+                      page_size=d.page_size, num_pages=max(d.num_pages, d2.num_pages), sm_scale=d.sm_scale,
+                      causal=d.causal)
+    tabs = [(x.qo_indptr.numpy(), x.kv_indptr.numpy(), x.kv_indices.numpy(), x.last_page_len.numpy()) for x in (d, d2)]
+
+    def host_us(fn, n=100):
+        t0 = time.perf_counter()
+        for i in range(n):
+            fn(i)
+        return (time.perf_counter() - t0) / n * 1e6
+
+    reuse_us = host_us(lambda i: M.mla_plan_update(plan, *tabs[0]))
+    replan_us = host_us(lambda i: M.mla_plan_update(plan, *tabs[i % 2]))
+
+    def fresh(i):
+        p = M.mla_plan(*tabs[i % 2], num_heads=d.num_heads, page_size=d.page_size,
+                       num_pages=max(d.num_pages, d2.num_pages), sm_scale=d.sm_scale, causal=d.causal)
+        p.destroy()
+
+    fresh_us = host_us(fresh)
+    torch.cuda.synchronize(device)
+    plan.destroy()
+    res["plan_reuse_decode_b64"] = {"unchanged_update_us": reuse_us, "changed_update_us": replan_us,
+                                    "fresh_plan_us": fresh_us,
+                                    "note": "host wall time per call, from numpy tables (binding included)"}
+    return res
 
 
 def reduce_max_over_ranks(x: float, dist, device) -> float:
@@ -498,6 +657,10 @@ def run_native(args):
                    "sample": f"first {rows} of {d.batch} rows of {args.workload} (all heads), fp64 NumPy "
                              f"oracle, {dt:.1f} s wall"}
 
+    next_rows = None
+    if rank == 0 and world == 1 and not args.no_next:
+        next_rows = measure_next_rows(device, peaks)
+
     attn_s = res["attn_ms"] * 1e-3
     traffic = kernel_traffic(args.workload)
     roofline = {
@@ -540,6 +703,7 @@ def run_native(args):
         "tflops": summ["tflops"],
         "frac_tensor": summ["frac_tensor"],
         "others": others,
+        "next_rows": next_rows,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -99,7 +99,9 @@ typedef struct {
    * all name its pages") attend that shared prefix together: one work item per 128
    * query rows of the whole group covers the prefix keys, its partial results are
    * merged by log-sum-exp with each row's own suffix.  Applies where the shared prefix
-   * spans at least MLA_KEY_TILE keys and every query of the group sees all of it.    */
+   * spans at least MLA_KEY_TILE keys, every query of the group sees all of it, and one
+   * prefix tile packs the query tiles of two or more rows (H * q_b <= 64): with 128
+   * heads a token already fills a tile, so a prefix tile would only add a merge.     */
   int32_t cascade;
 } mla_plan_options;
 

@@ -61,8 +61,9 @@ struct QTile {
 constexpr double kItemCost = 3.0;
 constexpr double kSplitCost = 2.0;
 
-// Longest-processing-time-first makespan of `costs` over `units` identical units.
-double lpt_makespan(std::vector<double> costs, int units) {
+// Longest-processing-time-first makespan of `costs` over `units` identical units.  Stops
+// early (returning a value >= `give_up`) once the makespan cannot end below `give_up`.
+double lpt_makespan(std::vector<double>& costs, int units, double give_up) {
   std::sort(costs.begin(), costs.end(), std::greater<double>());
   std::priority_queue<double, std::vector<double>, std::greater<double>> load;
   for (int i = 0; i < units; ++i) load.push(0.0);
@@ -72,6 +73,7 @@ double lpt_makespan(std::vector<double> costs, int units) {
     load.pop();
     l += c;
     worst = std::max(worst, l);
+    if (worst >= give_up) return worst;
     load.push(l);
   }
   return worst;
@@ -121,7 +123,8 @@ bool fits(const Counts& c, const PlanRequest& r) {
   return true;
 }
 
-double estimate(const std::vector<QTile>& tiles, int32_t chunk, int units) {
+double estimate(const std::vector<QTile>& tiles, int32_t chunk, int units,
+                double give_up = std::numeric_limits<double>::infinity()) {
   std::vector<double> costs;
   costs.reserve(tiles.size() * 2);
   int64_t partials = 0;
@@ -138,7 +141,8 @@ double estimate(const std::vector<QTile>& tiles, int32_t chunk, int units) {
     }
   }
   // The merge pass reads every partial once, spread over all units.
-  return lpt_makespan(costs, units) + kSplitCost * double(partials) / units;
+  const double merge = kSplitCost * double(partials) / units;
+  return lpt_makespan(costs, units, give_up - merge) + merge;
 }
 
 }  // namespace
@@ -288,10 +292,15 @@ mla_status build_layout(const PlanRequest& req, PlanLayout* out) {
             c.n_out = 0;
             while (o < o1 && c.n_rows + outs[o].n_rows <= kTileM) {
               c.n_rows += outs[o].n_rows;
-              out_cascaded[o] = true;
-              suffix_from[o] = static_cast<int32_t>(s);
               ++c.n_out;
               ++o;
+            }
+            // A prefix tile that serves a single output tile reads the same keys for the
+            // same queries as that tile would, and only adds a merge: leave it out.
+            if (c.n_out < 2) continue;
+            for (int32_t oo = c.first_out; oo < c.first_out + c.n_out; ++oo) {
+              out_cascaded[oo] = true;
+              suffix_from[oo] = static_cast<int32_t>(s);
             }
             c.page_base = kv_indptr[g];
             c.kv_len = static_cast<int32_t>(s);
@@ -334,19 +343,46 @@ mla_status build_layout(const PlanRequest& req, PlanLayout* out) {
     if (!fits(count_for(tiles, n_out, chunk), req)) return MLA_ERR_INVALID_ARGUMENT;
   } else {
     if (!fits(count_for(tiles, n_out, 0), req)) return MLA_ERR_INVALID_ARGUMENT;
-    if (req.split_keys == 0 && !tiles.empty() && max_ntiles > 1) {
-      double best = estimate(tiles, 0, units);
-      const double avg = (double(total_key_tiles) + kItemCost * tiles.size()) / units;
+    const double avg = (double(total_key_tiles) + kItemCost * tiles.size()) / units;
+    // No split can help when the longest tile already fits in the average load of a pair.
+    if (req.split_keys == 0 && !tiles.empty() && max_ntiles > 1 && max_ntiles + kItemCost > avg) {
       std::vector<int32_t> cands;
       for (int32_t dv = 2; dv <= 64; ++dv) cands.push_back((max_ntiles + dv - 1) / dv);
       for (double f : {1.0, 1.5, 2.0, 3.0, 4.0, 6.0, 8.0}) cands.push_back((int32_t)std::ceil(avg / f));
       std::sort(cands.begin(), cands.end(), std::greater<int32_t>());
       cands.erase(std::unique(cands.begin(), cands.end()), cands.end());
+      // Score every candidate by a lower bound on its makespan (the largest of: its
+      // longest item, its average load per pair, and the items some pair must take
+      // times the shortest item; plus the merge pass), then run the full LPT estimate
+      // on the few best.
+      std::vector<std::pair<double, int32_t>> scored;
       for (int32_t c : cands) {
         if (c < 2 || c >= max_ntiles) continue;
         if (!fits(count_for(tiles, n_out, c), req)) continue;
-        const double e = estimate(tiles, c, units);
-        if (e < best * 0.99) {  // prefer fewer splits unless clearly better
+        double longest = 0.0, shortest = std::numeric_limits<double>::infinity(), sum = 0.0, partials = 0.0;
+        int64_t items = 0;
+        for (const QTile& t : tiles) {
+          const int32_t n = pieces_for(t.ntiles, c);
+          const bool part = n > 1 || t.must_merge;
+          const double fixed = kItemCost + (part ? kSplitCost : 0.0);
+          longest = std::max(longest, double((t.ntiles + n - 1) / n) + fixed);
+          shortest = std::min(shortest, double(t.ntiles / n) + fixed);
+          sum += t.ntiles + n * fixed;
+          items += n;
+          if (part) partials += n;
+        }
+        const double per_unit = double((items + units - 1) / units) * shortest;
+        scored.emplace_back(std::max({longest, sum / units, per_unit}) + kSplitCost * partials / units, c);
+      }
+      std::sort(scored.begin(), scored.end());
+      double best = estimate(tiles, 0, units);
+      constexpr size_t kFullEstimates = 4;
+      for (size_t i = 0; i < scored.size() && i < kFullEstimates; ++i) {
+        const int32_t c = scored[i].second;
+        // (an estimate that cannot beat best * 0.99 stops early: prefer fewer splits
+        // unless clearly better)
+        const double e = estimate(tiles, c, units, best * 0.99);
+        if (e < best * 0.99) {
           best = e;
           chunk = c;
         }

@@ -273,7 +273,7 @@ def test_merge_state_matches_oracle_including_empty_states():
 
 
 # ------------------------------------------------------------------------- cascade
-@pytest.mark.parametrize("H,P,q", [(128, 64, 4), (16, 16, 4), (16, 16, 3), (64, 32, 1)])
+@pytest.mark.parametrize("H,P,q", [(16, 16, 4), (16, 16, 3), (64, 32, 1), (32, 64, 2)])
 def test_cascade_matches_oracle(H, P, q):
     B, group = 8, 4
     k = [1024 + q + 37 * i for i in range(B)]
@@ -288,14 +288,20 @@ def test_cascade_matches_oracle(H, P, q):
     plan.destroy()
 
 
+def spec_shapes_16_heads():
+    """The speculative shared-prefix workload's rows (128 rows, 4 queries, groups of 8
+    sharing their first 16 pages) with 16 query heads, where a prefix tile packs the
+    queries of two rows."""
+    t = make_config("spec_shared_prefix", tables_only=True)
+    return make_custom(t.q_lens, t.kv_lens, 16, 64, shared_group=8, shared_pages=16, seed=0,
+                       name="spec_shared_prefix_h16")
+
+
 @pytest.mark.slow
 def test_cascade_full_size_speculative_sampled():
-    """The speculative shared-prefix workload (128 rows, 4 queries each, groups of 8
-    sharing 1024 keys) with the cascade on, checked on sampled tokens."""
-    d = make_config("spec_shared_prefix")
+    d = spec_shapes_16_heads()
     plan = _plan(d, cascade=True)
-    info = M.mla_plan_get_info(plan)
-    assert info["num_cascade"] >= 16 * 32
+    assert M.mla_plan_get_info(plan)["num_cascade"] >= 16 * 4
     out, lse = M.mla_run(plan, d.q_nope.to(DEV), d.q_pe.to(DEV), d.cache.to(DEV), return_lse=True)
     assert M.mla_plan_check(plan) == M.MLA_OK
     qo = d.qo_indptr.numpy()

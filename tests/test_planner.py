@@ -184,24 +184,26 @@ def test_no_split_for_small_decode():
     assert desc["info"]["num_merge"] == 0 and desc["info"]["num_work"] == 2
 
 
-@pytest.mark.parametrize("H,P,q", [(128, 64, 4), (16, 16, 4), (16, 16, 3), (32, 32, 1), (64, 128, 2)])
+@pytest.mark.parametrize("H,P,q", [(128, 64, 4), (16, 16, 4), (16, 16, 3), (32, 32, 1), (64, 128, 2), (64, 64, 1)])
 def test_cascade_layout_covers_once_and_groups_rows(H, P, q):
     """Shared-prefix cascade (consecutive rows naming the same first pages attend them
-    together): coverage, visibility and merge references stay exact, and every group
-    with a long enough shared prefix gets prefix items spanning its rows' queries."""
-    B, group, shared = 12, 4, (1024 // P)
+    together): coverage, visibility and merge references stay exact; a group gets
+    prefix tiles exactly where one tile packs the queries of two or more rows."""
+    B, group = 12, 4
     k = [1024 + q + 13 * i for i in range(B)]
-    d = make_custom([q] * B, k, H, P, shared_group=group, shared_pages=shared, tables_only=True, seed=H + P)
+    d = make_custom([q] * B, k, H, P, shared_group=group, shared_pages=1024 // P, tables_only=True, seed=H + P)
     p = plan_tables(d, cascade=True)
     desc = M.mla_plan_describe(p)
     check_layout(d, desc)
     info = desc["info"]
-    # shared prefix keys = 1024 (a multiple of 64, visible in full to every query)
-    rows_per_item = min(128, max(H * q, (128 // (H * q)) * H * q))
-    expect_items = (B // group) * (-(-group * q * H // rows_per_item))
-    assert info["num_cascade"] >= expect_items
-    prefix = [w for w in desc["work"] if w[3] == 1024 and w[6] >= 1024]
-    assert len(prefix) >= expect_items
+    per_tile = 128 // (H * q) if H * q <= 128 else 1  # rows' query tiles per prefix tile
+    if per_tile < 2:
+        assert info["num_cascade"] == 0  # nothing to pack: the plan is the plain one
+    else:
+        tiles = (B // group) * (-(-group // per_tile))
+        prefix = [w for w in desc["work"] if w[6] >= w[3] and w[1] > H * q]
+        assert info["num_cascade"] >= tiles and len(prefix) >= tiles
+        assert all(w[1] <= 128 for w in prefix)
     # without the option, nothing is cascaded
     assert M.mla_plan_describe(plan_tables(d))["info"]["num_cascade"] == 0
 
