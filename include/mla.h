@@ -4,14 +4,15 @@
  * The operation (page "mstar.engine.resources.attn.flashinfer_mla": module
  * description, FlashInferMLAWrapper.plan / .run, FlashInferMLAManager.run):
  *
- *   The cache holds one latent row per token, [ckv (kv_lora_rank = 512) | kpe (64)],
- *   bf16, in pages of `page_size` tokens: cache[num_pages][page_size][576].
+ *   The cache holds one latent row per token, [ckv (kv_lora_rank = 512) | kpe (rope_dim
+ *   = 64, or 0)], bf16, in pages of `page_size` tokens: cache[num_pages][page_size][D],
+ *   D = 512 + rope_dim (576 for the DeepSeek shape).
  *   Row b of a batch names its pages by kv_indices[kv_indptr[b] .. kv_indptr[b+1]);
  *   its last page holds last_page_len[b] tokens, so it has
  *       k_b = (n_b - 1) * page_size + last_page_len[b]   keys   (0 if n_b == 0).
  *   Its query tokens are t in [qo_indptr[b], qo_indptr[b+1]), q_b of them, each
  *   with H heads of absorbed query q_nope[t][h][512] (already multiplied by W_UK)
- *   and rope query q_pe[t][h][64] (used as given: the library rotates nothing).
+ *   and rope query q_pe[t][h][rope_dim] (used as given: the library rotates nothing).
  *   For query i of row b (0-based) and causal = 1, the visible keys are
  *       j < vis = clamp(k_b - q_b + i + 1, 0, k_b)
  *   (queries aligned to the END of the keys: page
@@ -54,7 +55,7 @@ typedef enum {
 typedef struct {
   int32_t num_heads;    /* H: local query heads; 16, 32, 64 or 128                 */
   int32_t kv_lora_rank; /* ckv width; must be 512                                  */
-  int32_t rope_dim;     /* kpe width; must be 64                                   */
+  int32_t rope_dim;     /* kpe width: 64, or 0 (no rope part: q_pe is not read)   */
   int32_t page_size;    /* tokens per page; 16, 32, 64 or 128                      */
   int32_t num_pages;    /* pages in the cache pool (cache.shape[0]) , >= 1         */
   float sm_scale;       /* softmax scale applied to q.k; finite and > 0            */
@@ -132,8 +133,8 @@ typedef struct mla_plan_s* mla_plan_t; /* opaque ("immutable and opaque to runne
                                           FlashInferMLAManager.plan)                 */
 
 /* 1 if the library runs this shape on sm_100a, else 0.  The pages' kernel is
- * specialised to ckv 512 with kpe 0 or 64 (flashinfer_mla_supports); this library
- * implements kpe 64 only, H in {16, 32, 64, 128}, page_size in {16, 32, 64, 128}. */
+ * specialised to ckv 512 with kpe 0 or 64 (flashinfer_mla_supports); so is this
+ * library, with H in {16, 32, 64, 128} and page_size in {16, 32, 64, 128}. */
 int mla_supports(int kv_lora_rank, int rope_dim, int num_heads, int page_size);
 
 /* Build a plan for one step (FlashInferMLAWrapper.plan: "inputs may be CPU tensors").
@@ -160,8 +161,10 @@ mla_status mla_plan(const mla_dims* dims, int32_t batch, const int32_t* qo_indpt
 
 /* Run the attention of a plan (FlashInferMLAWrapper.run).
  *   q_nope  device bf16 [T][H][512], contiguous, 16-byte aligned
- *   q_pe    device bf16 [T][H][64], contiguous, 16-byte aligned
- *   cache   device bf16 [num_pages][page_size][576], contiguous, 16-byte aligned
+ *   q_pe    device bf16 [T][H][64], contiguous, 16-byte aligned (NULL allowed when
+ *           rope_dim is 0: it is not read)
+ *   cache   device bf16 [num_pages][page_size][512 + rope_dim], contiguous, 16-byte
+ *           aligned
  *   out     device bf16 [T][H][512], contiguous, 16-byte aligned (written)
  *   lse     device fp32 [T][H] or NULL (written when non-NULL)
  *   stream  cudaStream_t (may be NULL)
@@ -226,8 +229,10 @@ mla_status mla_plan_update(mla_plan_t plan, int32_t batch, const int32_t* qo_ind
  * before calling run").  Token i of row b (t = qo_indptr[b] + i) is key position
  * k_b - q_b + i of its row, i.e. slot (k_b - q_b + i) mod page_size of page
  * kv_indices[kv_indptr[b] + (k_b - q_b + i) / page_size]:
- *   kv_new  device bf16 [T][576] ([ckv | kpe] per token), contiguous, 16-byte aligned
- *   cache   device bf16 [num_pages][page_size][576] (written at those slots only)
+ *   kv_new  device bf16 [T][512 + rope_dim] ([ckv | kpe] per token), contiguous,
+ *           16-byte aligned
+ *   cache   device bf16 [num_pages][page_size][512 + rope_dim] (written at those slots
+ *           only)
  * One launch, no allocation, no synchronisation.  Two tokens naming the same slot (a
  * page listed twice) leave one of the two rows there.  Errors: INVALID_ARGUMENT (NULL
  * or misaligned pointer, or a row with q_b > k_b, whose tokens have no slots), CUDA. */

@@ -184,11 +184,13 @@ def mla_supports(kv_lora_rank: int, rope_dim: int, num_heads: int, page_size: in
 class MlaPlan:
     """Owns one C plan handle (``mla_plan_t``); destroyed with the object."""
 
-    def __init__(self, handle: int, batch: int, num_heads: int, total_tokens: int, graph_max_tokens: int = 0):
+    def __init__(self, handle: int, batch: int, num_heads: int, total_tokens: int, graph_max_tokens: int = 0,
+                 rope_dim: int = ROPE_DIM):
         self._h = ctypes.c_void_p(handle)
         self.batch = batch
         self.num_heads = num_heads
         self.total_tokens = total_tokens
+        self.rope_dim = rope_dim
         # a graph plan's per-token buffers hold graph_max_tokens tokens
         self.graph_max_tokens = graph_max_tokens
 
@@ -248,7 +250,8 @@ def mla_plan(qo_indptr, kv_indptr, kv_indices, last_page_len, *, num_heads: int,
                       1 if causal else 0, ctypes.c_void_p(stream or 0), ctypes.byref(opts), ctypes.byref(out))
     if st != MLA_OK:
         raise MlaError(st, "mla_plan")
-    return MlaPlan(out.value, batch, num_heads, int(qo[-1]), graph_max_tokens if graph_max_tokens > 0 else 0)
+    return MlaPlan(out.value, batch, num_heads, int(qo[-1]), graph_max_tokens if graph_max_tokens > 0 else 0,
+                   rope_dim)
 
 
 def mla_plan_update(plan: MlaPlan, qo_indptr, kv_indptr, kv_indices, last_page_len, stream=None) -> bool:
@@ -322,15 +325,18 @@ def _check_dev_tensor(t, name, dtype, shape):
 def mla_run(plan: MlaPlan, q_nope, q_pe, cache, out=None, lse=None, return_lse: bool = False, stream=None,
             kv_new=None):
     """Run the planned attention (``mla_run``).  Returns ``out`` or ``(out, lse)``.
-    With ``kv_new`` ([T, 576] bf16) the step's latent rows are first written into the
-    cache (``mla_run_append``)."""
+    With ``kv_new`` ([T, 512 + rope_dim] bf16) the step's latent rows are first written
+    into the cache (``mla_run_append``).  ``q_pe`` may be None for a plan with
+    ``rope_dim=0``."""
     import torch
 
-    T, H = plan.token_capacity, plan.num_heads
+    T, H, R = plan.token_capacity, plan.num_heads, plan.rope_dim
+    width = KV_LORA_RANK + R
     _check_dev_tensor(q_nope, "q_nope", torch.bfloat16, (T, H, KV_LORA_RANK))
-    _check_dev_tensor(q_pe, "q_pe", torch.bfloat16, (T, H, ROPE_DIM))
-    if cache.dim() != 3 or cache.shape[-1] != KV_LORA_RANK + ROPE_DIM:
-        raise ValueError("cache must be [num_pages, page_size, 576]")
+    if R > 0 or q_pe is not None:
+        _check_dev_tensor(q_pe, "q_pe", torch.bfloat16, (T, H, R))
+    if cache.dim() != 3 or cache.shape[-1] != width:
+        raise ValueError(f"cache must be [num_pages, page_size, {width}]")
     _check_dev_tensor(cache, "cache", torch.bfloat16, tuple(cache.shape))
     if out is None:
         out = torch.empty((T, H, KV_LORA_RANK), dtype=torch.bfloat16, device=q_nope.device)
@@ -340,18 +346,19 @@ def mla_run(plan: MlaPlan, q_nope, q_pe, cache, out=None, lse=None, return_lse: 
     if lse is not None:
         _check_dev_tensor(lse, "lse", torch.float32, (T, H))
     if kv_new is not None:
-        _check_dev_tensor(kv_new, "kv_new", torch.bfloat16, (T, KV_LORA_RANK + ROPE_DIM))
+        _check_dev_tensor(kv_new, "kv_new", torch.bfloat16, (T, width))
     if stream is None:
         stream = torch.cuda.current_stream(q_nope.device).cuda_stream
     lib = load_library()
     lse_p = ctypes.c_void_p(lse.data_ptr() if lse is not None else 0)
+    qpe_p = ctypes.c_void_p(q_pe.data_ptr() if q_pe is not None else 0)
     if kv_new is None:
-        st = lib.mla_run(plan.handle, ctypes.c_void_p(q_nope.data_ptr()), ctypes.c_void_p(q_pe.data_ptr()),
+        st = lib.mla_run(plan.handle, ctypes.c_void_p(q_nope.data_ptr()), qpe_p,
                          ctypes.c_void_p(cache.data_ptr()), ctypes.c_void_p(out.data_ptr()), lse_p,
                          ctypes.c_void_p(stream or 0))
         what = "mla_run"
     else:
-        st = lib.mla_run_append(plan.handle, ctypes.c_void_p(q_nope.data_ptr()), ctypes.c_void_p(q_pe.data_ptr()),
+        st = lib.mla_run_append(plan.handle, ctypes.c_void_p(q_nope.data_ptr()), qpe_p,
                                 ctypes.c_void_p(kv_new.data_ptr()), ctypes.c_void_p(cache.data_ptr()),
                                 ctypes.c_void_p(out.data_ptr()), lse_p, ctypes.c_void_p(stream or 0))
         what = "mla_run_append"
@@ -365,9 +372,10 @@ def mla_append_kv(plan: MlaPlan, kv_new, cache, stream=None) -> None:
     (``mla_append_kv``)."""
     import torch
 
-    _check_dev_tensor(kv_new, "kv_new", torch.bfloat16, (plan.token_capacity, KV_LORA_RANK + ROPE_DIM))
-    if cache.dim() != 3 or cache.shape[-1] != KV_LORA_RANK + ROPE_DIM:
-        raise ValueError("cache must be [num_pages, page_size, 576]")
+    width = KV_LORA_RANK + plan.rope_dim
+    _check_dev_tensor(kv_new, "kv_new", torch.bfloat16, (plan.token_capacity, width))
+    if cache.dim() != 3 or cache.shape[-1] != width:
+        raise ValueError(f"cache must be [num_pages, page_size, {width}]")
     _check_dev_tensor(cache, "cache", torch.bfloat16, tuple(cache.shape))
     if stream is None:
         stream = torch.cuda.current_stream(kv_new.device).cuda_stream
@@ -439,7 +447,8 @@ def mla_run_noalloc(qo_indptr, kv_indptr, kv_indices, last_page_len, q_nope, q_p
         raise MlaError(MLA_ERR_INVALID_ARGUMENT, "mla_run_noalloc: table lengths")
     T = int(qo[-1])
     _check_dev_tensor(q_nope, "q_nope", torch.bfloat16, (T, num_heads, kv_lora_rank))
-    _check_dev_tensor(q_pe, "q_pe", torch.bfloat16, (T, num_heads, rope_dim))
+    if rope_dim > 0 or q_pe is not None:
+        _check_dev_tensor(q_pe, "q_pe", torch.bfloat16, (T, num_heads, rope_dim))
     _check_dev_tensor(cache, "cache", torch.bfloat16, tuple(cache.shape))
     _check_dev_tensor(out, "out", torch.bfloat16, (T, num_heads, kv_lora_rank))
     if lse is not None:
@@ -450,7 +459,8 @@ def mla_run_noalloc(qo_indptr, kv_indptr, kv_indices, last_page_len, q_nope, q_p
     kvi_arr = kvi if len(kvi) else np.zeros(1, dtype=np.int32)
     st = load_library().mla_run_noalloc(
         ctypes.byref(dims), batch, _ptr(qo), _ptr(kvp), _ptr(kvi_arr), _ptr(last), 1 if causal else 0,
-        ctypes.c_void_p(q_nope.data_ptr()), ctypes.c_void_p(q_pe.data_ptr()), ctypes.c_void_p(cache.data_ptr()),
+        ctypes.c_void_p(q_nope.data_ptr()), ctypes.c_void_p(q_pe.data_ptr() if q_pe is not None else 0),
+        ctypes.c_void_p(cache.data_ptr()),
         ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(lse.data_ptr() if lse is not None else 0),
         ctypes.c_void_p(stream or 0))
     if st != MLA_OK:

@@ -350,8 +350,9 @@ inline bool misaligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x)
 // Shared checks and parameter set-up of the attention launch.
 mla_status attention_launch_of(mla_plan_t p, const void* q_nope, const void* q_pe, const void* cache, void* out,
                                float* lse, AttnLaunch* a) {
-  if (!q_nope || !q_pe || !cache || !out) return MLA_ERR_INVALID_ARGUMENT;
-  if (misaligned16(q_nope) || misaligned16(q_pe) || misaligned16(cache) || misaligned16(out) ||
+  const bool rope = p->dims.rope_dim > 0;  // without kpe, q_pe is not read (may be NULL)
+  if (!q_nope || (rope && !q_pe) || !cache || !out) return MLA_ERR_INVALID_ARGUMENT;
+  if (misaligned16(q_nope) || (rope && misaligned16(q_pe)) || misaligned16(cache) || misaligned16(out) ||
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return MLA_ERR_INVALID_ARGUMENT;
   AttnParams& ap = a->p;
@@ -366,6 +367,7 @@ mla_status attention_launch_of(mla_plan_t p, const void* q_nope, const void* q_p
   ap.scale_log2 = p->dims.sm_scale * 1.4426950408889634f;
   ap.num_heads = p->dims.num_heads;
   ap.page_size = p->dims.page_size;
+  ap.rope_dim = p->dims.rope_dim;
   ap.timeout_ns = p->opts.wait_timeout_ns ? p->opts.wait_timeout_ns : 4000000000ull;
   ap.debug_flags = p->opts.debug_flags;
   a->q_nope = q_nope;
@@ -390,6 +392,7 @@ mla_status append_launch_of(mla_plan_t p, const void* kv_new, void* cache, Appen
   ap->rows = p->d_append();
   ap->src = kv_new;
   ap->cache = cache;
+  ap->width = kCkv + p->dims.rope_dim;
   *n_tokens = static_cast<int>(p->sz.cap_tokens);
   return MLA_OK;
 }

@@ -132,9 +132,8 @@ __device__ __forceinline__ void record_error(int32_t* status, int32_t site) {
 //   softmax  : S(j) = ours + peer's; mask, online softmax, P(j) -> P[j % 2]
 //   PV warp  : PV(j): O += P[j % 2] . V(stage j % 3), as soon as P(j) is written
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
-    mla_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qpe,
-                    const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_kpe,
-                    const AttnParams p) {
+    mla_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                    const __grid_constant__ CUtensorMap tm_kpe, const AttnParams p) {
   using namespace attn;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
@@ -179,9 +178,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   }
   if (warp == kWarpProducer && lane == 0) {
     tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_qpe);
     tma_prefetch_desc(&tm_kv);
-    tma_prefetch_desc(&tm_kpe);
+    if (p.rope_dim > 0) tma_prefetch_desc(&tm_kpe);
   }
   if (warp == kWarpMma) {
     tmem_alloc(smem_addr(tmem_slot), kTmemCols);
@@ -239,14 +237,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         if (j >= kStages && !wait_warp(bar(bKVEmpty + st), ((j / kStages) - 1) & 1, kSiteProducer, false)) break;
         if ((p.debug_flags & MLA_DEBUG_DROP_FIRST_KV_LOAD) && j == 0) continue;
         const uint32_t dst = sb + kKV + st * kStageBytes;
-        if (lane == 0) mbar_arrive_expect_tx(bar(bKVFull + st), kStageBytes);
+        if (lane == 0) mbar_arrive_expect_tx(bar(bKVFull + st), p.rope_dim > 0 ? kStageBytes : kStageKpe);
         for (int b = 0; b < nbox; ++b) {
           const int key0 = w.key_begin + kTileN * j + b * BR;
           const int row = page_of(key0 / P) * P + (key0 % P);
           if (lane == 0) {
             for (int c = 0; c < 4; ++c)
               tma_load_2d(dst + c * 8192 + b * BR * 128, &tm_kv, bar(bKVFull + st), 256 * rank + 64 * c, row);
-            tma_load_2d(dst + kStageKpe + b * BR * 64, &tm_kpe, bar(bKVFull + st), kCkv + 32 * rank, row);
+            if (p.rope_dim > 0)
+              tma_load_2d(dst + kStageKpe + b * BR * 64, &tm_kpe, bar(bKVFull + st), kCkv + 32 * rank, row);
           }
         }
         last_issued[st] = j;
@@ -297,10 +296,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
             const uint64_t bd = smem_desc(kv + 3 * 8192 + s * 32, 16, 1024, 2);
             mma_ts(scol, tmem + kColQ + 8 * s, bd, id_qk, 1u);
           }
-          for (int s = 0; s < 2; ++s) {  // kpe: A from TMEM
-            const uint64_t bd = smem_desc(kv + kStageKpe + s * 32, 16, 512, 4);
-            mma_ts(scol, tmem + kColQpe + 8 * s, bd, id_qk, 1u);
-          }
+          if (p.rope_dim > 0)
+            for (int s = 0; s < 2; ++s) {  // kpe: A from TMEM
+              const uint64_t bd = smem_desc(kv + kStageKpe + s * 32, 16, 512, 4);
+              mma_ts(scol, tmem + kColQpe + 8 * s, bd, id_qk, 1u);
+            }
           mma_commit(bar(bSFull + b2));
         }
         __syncwarp();
@@ -391,17 +391,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       if (r < w.n_rows) {
         const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q_nope) +
                                                           static_cast<size_t>(w.q_row0 + r) * kCkv + 256 * rank + 192);
-        const uint4* srp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q_pe) +
-                                                          static_cast<size_t>(w.q_row0 + r) * kRope + 32 * rank);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const uint4 v = __ldg(src + i);
           qa[4 * i] = v.x; qa[4 * i + 1] = v.y; qa[4 * i + 2] = v.z; qa[4 * i + 3] = v.w;
         }
+        if (p.rope_dim > 0) {
+          const uint4* srp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q_pe) +
+                                                            static_cast<size_t>(w.q_row0 + r) * kRope + 32 * rank);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint4 v = __ldg(srp + i);
-          qb[4 * i] = v.x; qb[4 * i + 1] = v.y; qb[4 * i + 2] = v.z; qb[4 * i + 3] = v.w;
+          for (int i = 0; i < 4; ++i) {
+            const uint4 v = __ldg(srp + i);
+            qb[4 * i] = v.x; qb[4 * i + 1] = v.y; qb[4 * i + 2] = v.z; qb[4 * i + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) qb[i] = 0u;
         }
       } else {
 #pragma unroll
@@ -711,14 +716,20 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
   p.nan_guard = __builtin_nanf("");
   p.box_rows = p.page_size < kTileN ? p.page_size : kTileN;
   const uint32_t br = static_cast<uint32_t>(p.box_rows);
-  CUtensorMap tm_q, tm_qpe, tm_kv, tm_kpe;
+  // the cache row is [ckv 512 | kpe rope_dim]; without kpe the kpe map is never used
+  const uint64_t width = static_cast<uint64_t>(kCkv + p.rope_dim);
+  CUtensorMap tm_q, tm_kv, tm_kpe;
   if (!encode_2d(&tm_q, a.q_nope, a.rows, kCkv, 64, kTileM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_2d(&tm_qpe, a.q_pe, a.rows, kRope, 32, kTileM, CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !encode_2d(&tm_kv, a.cache, a.cache_rows, kLatent, 64, br, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_2d(&tm_kpe, a.cache, a.cache_rows, kLatent, 32, br, CU_TENSOR_MAP_SWIZZLE_64B))
+      !encode_2d(&tm_kv, a.cache, a.cache_rows, width, 64, br, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+  if (p.rope_dim > 0) {
+    if (!encode_2d(&tm_kpe, a.cache, a.cache_rows, width, 32, br, CU_TENSOR_MAP_SWIZZLE_64B))
+      return cudaErrorInvalidValue;
+  } else {
+    tm_kpe = tm_kv;
+  }
   if (!a.wait_prior_grid) {
-    mla_attn_kernel<<<2 * a.num_work, attn::kThreads, attn::kSmemAlloc, stream>>>(tm_q, tm_qpe, tm_kv, tm_kpe, p);
+    mla_attn_kernel<<<2 * a.num_work, attn::kThreads, attn::kSmemAlloc, stream>>>(tm_q, tm_kv, tm_kpe, p);
     return cudaGetLastError();
   }
   // Programmatic dependent of the append: set-up and query loads overlap it.
@@ -732,7 +743,7 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, mla_attn_kernel, tm_q, tm_qpe, tm_kv, tm_kpe, p);
+  return cudaLaunchKernelEx(&cfg, mla_attn_kernel, tm_q, tm_kv, tm_kpe, p);
 }
 
 cudaError_t launch_merge(const MergeParams& p, int num_merge, cudaStream_t stream) {

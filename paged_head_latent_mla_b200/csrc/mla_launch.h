@@ -15,7 +15,7 @@ struct AttnParams {
   const WorkItem* work;
   const int32_t* kv_indices;
   const void* q_nope;  // bf16 [T*H, 512] (the kernel reads part of Q directly)
-  const void* q_pe;    // bf16 [T*H, 64]
+  const void* q_pe;    // bf16 [T*H, 64]; unused when rope_dim == 0
   void* out;         // bf16 [T*H, 512]
   float* lse;        // fp32 [T*H] or nullptr
   void* ws_o;        // bf16 [partials, 128, 512]
@@ -27,6 +27,7 @@ struct AttnParams {
   int32_t num_heads;
   int32_t page_size;
   int32_t box_rows;  // rows per KV box: min(page_size, 64)
+  int32_t rope_dim;  // kpe width: 64, or 0 (cache rows are then 512 wide)
   uint64_t timeout_ns;
   int32_t debug_flags;
 };
@@ -36,8 +37,8 @@ struct AttnParams {
 struct AttnLaunch {
   AttnParams p;
   const void* q_nope;   // bf16 [rows, 512]
-  const void* q_pe;     // bf16 [rows, 64]
-  const void* cache;    // bf16 [cache_rows, 576]
+  const void* q_pe;     // bf16 [rows, 64] (null when rope_dim == 0)
+  const void* cache;    // bf16 [cache_rows, 512 + rope_dim]
   uint64_t rows;        // T * H
   uint64_t cache_rows;  // num_pages * page_size
   int num_work;         // launch slots (CTA pairs)
@@ -57,8 +58,9 @@ struct MergeParams {
 // Latent-cache append: token t's row of src goes to cache row rows[t] (skipped if < 0).
 struct AppendParams {
   const int32_t* rows;  // [tokens]
-  const void* src;      // bf16 [tokens, 576]
-  void* cache;          // bf16 [cache_rows, 576]
+  const void* src;      // bf16 [tokens, width]
+  void* cache;          // bf16 [cache_rows, width]
+  int32_t width;        // 512 + rope_dim
 };
 
 // Merge of two attention states by their log-sum-exps.

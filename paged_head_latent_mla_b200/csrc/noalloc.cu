@@ -184,9 +184,10 @@ extern "C" mla_status mla_run_noalloc(const mla_dims* dims, int32_t batch, const
                              g_dev[dev].num_sms, &n_work, &n_merge, &n_refs, &n_ws_rows, &T);
   if (st != MLA_OK) return st;
   if (n_work == 0) return MLA_OK;
-  if (!q_nope || !q_pe || !cache || !out) return MLA_ERR_INVALID_ARGUMENT;
+  const bool rope = dims->rope_dim > 0;  // without kpe, q_pe is not read (may be NULL)
+  if (!q_nope || (rope && !q_pe) || !cache || !out) return MLA_ERR_INVALID_ARGUMENT;
   auto misaligned = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) != 0; };
-  if (misaligned(q_nope) || misaligned(q_pe) || misaligned(cache) || misaligned(out) ||
+  if (misaligned(q_nope) || (rope && misaligned(q_pe)) || misaligned(cache) || misaligned(out) ||
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return MLA_ERR_INVALID_ARGUMENT;
 
@@ -221,6 +222,7 @@ extern "C" mla_status mla_run_noalloc(const mla_dims* dims, int32_t batch, const
   ap.scale_log2 = dims->sm_scale * 1.4426950408889634f;
   ap.num_heads = dims->num_heads;
   ap.page_size = dims->page_size;
+  ap.rope_dim = dims->rope_dim;
   ap.timeout_ns = 4000000000ull;
   ap.debug_flags = 0;
   a.q_nope = q_nope;

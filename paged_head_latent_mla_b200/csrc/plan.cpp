@@ -20,7 +20,8 @@
 namespace mla {
 
 bool shape_supported(int kv_lora_rank, int rope_dim, int num_heads, int page_size) {
-  if (kv_lora_rank != kCkv || rope_dim != kRope) return false;
+  // ckv 512 with kpe 64 or 0 (flashinfer_mla_supports: "ckv 512, kpe 0 or 64")
+  if (kv_lora_rank != kCkv || (rope_dim != kRope && rope_dim != 0)) return false;
   if (num_heads != 16 && num_heads != 32 && num_heads != 64 && num_heads != 128) return false;
   if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128) return false;
   return true;

@@ -3,10 +3,10 @@
 //
 // Append (page "mstar.engine.resources.attn.base", AttentionManager.requires_kv_write:
 // a layer writes the step's K/V through the KV resource before calling run): every
-// token's 576-wide [ckv | kpe] row is copied to the cache row the plan assigned it.
-// The copy is HBM-bound: 1152 B read and 1152 B written per token, moved as 16-byte
-// vectors, 72 consecutive threads per token so that each token row is one contiguous
-// access on both sides.
+// token's [ckv | kpe] row (576 wide, or 512 without kpe) is copied to the cache row the
+// plan assigned it.  The copy is HBM-bound: 1152 B (1024 B) read and written per token,
+// moved as 16-byte vectors, one thread per vector and consecutive threads along a row,
+// so that each token row is one contiguous access on both sides.
 //
 // Merge (page "mstar.engine.resources.attn.flashinfer_mla", FlashInferMLAManager.run:
 // the log-sum-exp is returned for merging with another key segment): two states over
@@ -24,21 +24,23 @@ namespace mla {
 
 namespace {
 
-constexpr int kRowChunks = kLatent * 2 / 16;  // 16-byte pieces per cache row (72)
-constexpr int kAppendThreads = 4 * kRowChunks;  // 4 tokens per block
+constexpr int kMaxRowChunks = kLatent * 2 / 16;  // 16-byte pieces per cache row (72, or 64)
+constexpr int kAppendTokens = 4;                 // tokens per block
 
-__global__ void __launch_bounds__(kAppendThreads) mla_append_kernel(const AppendParams p, int num_tokens) {
+__global__ void __launch_bounds__(kAppendTokens * kMaxRowChunks) mla_append_kernel(const AppendParams p,
+                                                                                    int num_tokens) {
   // The attention launched after this grid as its programmatic dependent may start its
   // set-up now; its key loads wait for this grid to finish.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int t = blockIdx.x * 4 + threadIdx.x / kRowChunks;
-  const int c = threadIdx.x % kRowChunks;
+  const int chunks = p.width / 8;  // blockDim.x == kAppendTokens * chunks
+  const int t = blockIdx.x * kAppendTokens + threadIdx.x / chunks;
+  const int c = threadIdx.x % chunks;
   if (t >= num_tokens) return;
   const int32_t row = p.rows[t];
   if (row < 0) return;  // an empty slot of a graph plan
-  const uint4 v = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.src) +
-                                                 static_cast<size_t>(t) * kLatent * 2)[c];
-  reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.cache) + static_cast<size_t>(row) * kLatent * 2)[c] = v;
+  const size_t row_bytes = static_cast<size_t>(p.width) * 2;
+  const uint4 v = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.src) + t * row_bytes)[c];
+  reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.cache) + static_cast<size_t>(row) * row_bytes)[c] = v;
 }
 
 // One warp per row; lane l owns columns [16l, 16l + 16).
@@ -85,7 +87,9 @@ __global__ void __launch_bounds__(256) mla_merge_state_kernel(const MergeStatePa
 
 cudaError_t launch_append(const AppendParams& p, int num_tokens, cudaStream_t stream) {
   if (num_tokens <= 0) return cudaSuccess;
-  mla_append_kernel<<<(num_tokens + 3) / 4, kAppendThreads, 0, stream>>>(p, num_tokens);
+  if (p.width != kCkv && p.width != kLatent) return cudaErrorInvalidValue;
+  const int threads = kAppendTokens * (p.width / 8);
+  mla_append_kernel<<<(num_tokens + kAppendTokens - 1) / kAppendTokens, threads, 0, stream>>>(p, num_tokens);
   return cudaGetLastError();
 }
 

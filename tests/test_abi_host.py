@@ -46,7 +46,8 @@ def test_supports_matrix():
     for H in (16, 32, 64, 128):
         for P in (16, 32, 64, 128):
             assert M.mla_supports(512, 64, H, P)
-    assert not M.mla_supports(512, 0, 128, 64)  # kpe 0 is not implemented here
+    assert M.mla_supports(512, 0, 128, 64)  # kpe 0 or 64 (flashinfer_mla_supports)
+    assert not M.mla_supports(512, 32, 128, 64)
     assert not M.mla_supports(256, 64, 128, 64)
     assert not M.mla_supports(512, 64, 8, 64)
     assert not M.mla_supports(512, 64, 128, 1)
@@ -97,7 +98,7 @@ def test_invalid_arguments(bad):
 
 
 @pytest.mark.parametrize("bad", [dict(num_heads=8), dict(page_size=8), dict(kv_lora_rank=256),
-                                 dict(rope_dim=0), dict(num_heads=96)])
+                                 dict(rope_dim=32), dict(num_heads=96)])
 def test_unsupported_shapes(bad):
     with pytest.raises(M.MlaError) as e:
         _plan(**bad)

@@ -310,3 +310,46 @@ def test_cascade_full_size_speculative_sampled():
                                    d.last_page_len, d.page_size, d.sm_scale, causal=True, tokens=toks)
     _check(out, lse, ref_o, ref_l, rows=np.asarray(toks))
     plan.destroy()
+
+
+# ------------------------------------------------------------------------- kpe width 0
+def _no_rope(d):
+    """The same inputs without a rope part: cache rows 512 wide, no q_pe."""
+    return d.cache[..., :512].contiguous()
+
+
+@pytest.mark.parametrize("H,P,split", [(128, 64, 0), (16, 16, 128), (64, 32, 0), (128, 128, 256)])
+def test_kpe0_matches_oracle(H, P, split):
+    d = make_custom([1, 5, 0, 33, 2], [700, 130, 50, 2000, 3], H, P, seed=101 + H + P)
+    c512 = _no_rope(d)
+    plan = M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=H, page_size=P,
+                      num_pages=d.num_pages, sm_scale=d.sm_scale, causal=True, rope_dim=0, split_keys=split,
+                      wait_timeout_ns=TIMEOUT_NS)
+    out, lse = M.mla_run(plan, d.q_nope.to(DEV), None, c512.to(DEV), return_lse=True)
+    assert M.mla_plan_check(plan) == M.MLA_OK
+    ref_o, ref_l = O.mla_attention(d.q_nope, d.q_pe[..., :0], c512, d.qo_indptr, d.kv_indptr, d.kv_indices,
+                                   d.last_page_len, P, d.sm_scale, causal=True)
+    _check(out, lse, ref_o, ref_l)
+    # the append writes 512-wide rows
+    kv_new = _kv_new(int(d.qo_indptr[-1]), 102)[:, :512].contiguous()
+    cache = c512.to(DEV)
+    M.mla_append_kv(plan, kv_new.to(DEV), cache)
+    torch.cuda.synchronize()
+    ref = O.append_latent(c512, kv_new, d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, P)
+    assert torch.equal(cache.cpu(), torch.from_numpy(ref).to(torch.bfloat16))
+    plan.destroy()
+
+
+def test_kpe0_is_bitwise_the_rope_kernel_with_zero_q_pe():
+    """The rope kernel with q_pe = 0 adds exact zeros to every score, so its outputs are
+    bit-identical to the kernel without a rope part."""
+    d = make_custom([1, 4, 1], [3000, 200, 64], 128, 64, seed=103)
+    p64 = _plan(d)
+    o64, l64 = M.mla_run(p64, d.q_nope.to(DEV), torch.zeros_like(d.q_pe).to(DEV), d.cache.to(DEV), return_lse=True)
+    p0 = M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=128, page_size=64,
+                    num_pages=d.num_pages, sm_scale=d.sm_scale, causal=True, rope_dim=0, wait_timeout_ns=TIMEOUT_NS)
+    o0, l0 = M.mla_run(p0, d.q_nope.to(DEV), None, _no_rope(d).to(DEV), return_lse=True)
+    assert M.mla_plan_check(p64) == M.MLA_OK and M.mla_plan_check(p0) == M.MLA_OK
+    assert torch.equal(o0, o64) and torch.equal(l0, l64)
+    p64.destroy()
+    p0.destroy()

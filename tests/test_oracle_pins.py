@@ -347,6 +347,24 @@ def check_context_only_merge(oracle):
                              [2], P, SCALE, context_only=True)
 
 
+def check_kpe_zero_width(oracle):
+    """Without a rope part (kpe width 0, flashinfer_mla_supports: kpe 0 or 64) the scores
+    are q_nope . ckv alone: the same as the 576-wide form with q_pe = 0, whatever kpe
+    holds; the output is still built from the 512 ckv columns."""
+    d = _paged([3, 1, 5], [40, 70, 5], 2, 16, seed=31)
+    z = np.zeros_like(d["q_pe"])
+    o64, l64 = oracle.mla_attention(d["q_nope"], z, d["cache"], d["qo_indptr"], d["kv_indptr"], d["kv_indices"],
+                                    d["last_page_len"], 16, SCALE)
+    c512 = d["cache"][..., :D_C].copy()
+    o0, l0 = oracle.mla_attention(d["q_nope"], d["q_pe"][..., :0], c512, d["qo_indptr"], d["kv_indptr"],
+                                  d["kv_indices"], d["last_page_len"], 16, SCALE)
+    assert np.allclose(o0, o64, rtol=0, atol=1e-13) and np.allclose(l0, l64, rtol=0, atol=1e-13)
+    # and it differs from the rope form once q_pe is not zero
+    o1, _ = oracle.mla_attention(d["q_nope"], d["q_pe"], d["cache"], d["qo_indptr"], d["kv_indptr"],
+                                 d["kv_indices"], d["last_page_len"], 16, SCALE)
+    assert not np.allclose(o1, o0, atol=1e-6)
+
+
 ALL_CHECKS = [
     check_absorbed_equals_explicit,
     check_against_sdpa,
@@ -360,6 +378,7 @@ ALL_CHECKS = [
     check_kv_lengths,
     check_append_slots,
     check_context_only_merge,
+    check_kpe_zero_width,
 ]
 
 
