@@ -350,57 +350,96 @@ def time_workload(d, device, steps, warmup, dist=None, soak_s=0.0, sampler=None,
 
 
 def time_e2e(d, device, steps, warmup):
-    """The public API end to end with host buffers: per step, plan from host tables
-    (uploads the work lists and page table), copy the step's queries from pinned host
-    memory, run, read the result back to pinned host memory, check status."""
+    """The public API end to end with host buffers.  Every step plans from host tables
+    (mla_plan: uploads the work lists and page table), copies the step's queries from
+    pinned host memory, runs, and copies out/lse back to pinned host memory.  Steps are
+    pipelined two deep the way a serving loop overlaps them: step i's queries go up on a
+    copy stream while step i-1 computes, and step i-1's result comes down on another
+    while step i computes (separate device buffers per step parity).  Each plan's status
+    is read when it is retired, two steps later.  The timed region covers `steps`
+    complete steps, from before the first plan to the last result on the host, on the
+    device clock."""
     import torch
 
     import paged_head_latent_mla_b200 as M
 
+    T, H = d.total_tokens, d.num_heads
+    cache = d.cache.to(device)  # the KV cache is resident state, written by earlier steps
     qn_h = d.q_nope.pin_memory()
     qp_h = d.q_pe.pin_memory()
-    cache = d.cache.to(device)  # the KV cache is resident state, written by earlier steps
-    qn = torch.empty_like(qn_h, device=device)
-    qp = torch.empty_like(qp_h, device=device)
-    T, H = d.total_tokens, d.num_heads
-    out = torch.empty((T, H, 512), dtype=torch.bfloat16, device=device)
-    lse = torch.empty((T, H), dtype=torch.float32, device=device) if d.return_lse else None
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory() if lse is not None else None
+    bufs = []
+    for _ in range(2):
+        bufs.append({
+            "qn": torch.empty_like(qn_h, device=device),
+            "qp": torch.empty_like(qp_h, device=device),
+            "out": torch.empty((T, H, 512), dtype=torch.bfloat16, device=device),
+            "lse": torch.empty((T, H), dtype=torch.float32, device=device) if d.return_lse else None,
+            "out_h": torch.empty((T, H, 512), dtype=torch.bfloat16).pin_memory(),
+            "lse_h": torch.empty((T, H), dtype=torch.float32).pin_memory() if d.return_lse else None,
+            "uploaded": torch.cuda.Event(), "computed": torch.cuda.Event(), "downloaded": torch.cuda.Event(),
+        })
+    s_up, s_run, s_down = torch.cuda.Stream(device), torch.cuda.Stream(device), torch.cuda.Stream(device)
     h2d = [0]
+    live = []  # (plan) of steps not yet retired
 
-    def one():
-        plan = M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=H,
-                          page_size=d.page_size, num_pages=d.num_pages, sm_scale=d.sm_scale, causal=d.causal)
-        info = M.mla_plan_get_info(plan)
-        qn.copy_(qn_h, non_blocking=True)
-        qp.copy_(qp_h, non_blocking=True)
-        M.mla_run(plan, qn, qp, cache, out=out, lse=lse)
-        out_h.copy_(out, non_blocking=True)
-        if lse is not None:
-            lse_h.copy_(lse, non_blocking=True)
-        st = M.mla_plan_check(plan)  # synchronises and reads the 4-byte status word
+    def retire(plan):
+        st = M.mla_plan_check(plan)  # waits for that step's launches, reads its status word
         if st != 0:
             raise M.MlaError(st, "e2e")
+        plan.destroy()
+
+    def one(i):
+        b = bufs[i % 2]
+        plan = M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=H,
+                          page_size=d.page_size, num_pages=d.num_pages, sm_scale=d.sm_scale, causal=d.causal,
+                          stream=s_run.cuda_stream)
+        info = M.mla_plan_get_info(plan)
+        with torch.cuda.stream(s_up):
+            s_up.wait_event(b["computed"])  # step i-2 has finished reading these buffers
+            b["qn"].copy_(qn_h, non_blocking=True)
+            b["qp"].copy_(qp_h, non_blocking=True)
+            b["uploaded"].record(s_up)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(b["uploaded"])
+            s_run.wait_event(b["downloaded"])  # step i-2's result has left `out`
+            M.mla_run(plan, b["qn"], b["qp"], cache, out=b["out"], lse=b["lse"], stream=s_run.cuda_stream)
+            b["computed"].record(s_run)
+        with torch.cuda.stream(s_down):
+            s_down.wait_event(b["computed"])
+            b["out_h"].copy_(b["out"], non_blocking=True)
+            if b["lse"] is not None:
+                b["lse_h"].copy_(b["lse"], non_blocking=True)
+            b["downloaded"].record(s_down)
+        live.append(plan)
+        if len(live) > 2:
+            retire(live.pop(0))
         # work list, merge list and references, append rows, page table
         plan_bytes = (32 * info["num_work"] + 16 * info["num_merge"] + 4 * info["num_merge_refs"] + 4 * T +
                       4 * int(d.kv_indptr[-1]))
         h2d[0] = plan_bytes + qn_h.numel() * 2 + qp_h.numel() * 2
-        plan.destroy()
 
-    for _ in range(warmup):
-        one()
+    for i in range(warmup):
+        one(i)
+    while live:
+        retire(live.pop(0))
     torch.cuda.synchronize(device)
+    # device clock: from an event the compute stream passes before the first step is
+    # planned to one the download stream passes after the last result reached the host
+    # (host planning time shows up as device idle time inside the span)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        one()
-    e1.record()
-    torch.cuda.synchronize(device)
+    e0.record(s_run)
+    for i in range(steps):
+        one(i)
+    for b in bufs:
+        s_down.wait_event(b["downloaded"])
+    e1.record(s_down)
+    e1.synchronize()
+    while live:
+        retire(live.pop(0))
     ms = e0.elapsed_time(e1) / steps
-    d2h = out_h.numel() * 2 + (lse_h.numel() * 4 if lse_h is not None else 0) + 4
-    del cache
+    d2h = T * H * 512 * 2 + (T * H * 4 if d.return_lse else 0) + 4
+    del cache, bufs
     torch.cuda.empty_cache()
     return ms, h2d[0], d2h
 
@@ -637,7 +676,10 @@ def run_native(args):
         e2e_ms = reduce_max_over_ranks(e2e_ms, dist, device)
         e2e = {"value": job_throughput(w["kv_bytes"], world, e2e_ms), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms,
-               "includes": "mla_plan from host tables + H2D of queries + mla_run + D2H of out/lse + status read"}
+               "includes": "per step: mla_plan from host tables + H2D of queries from pinned memory + mla_run "
+                           "+ D2H of out/lse to pinned memory; steps pipelined two deep on separate copy and "
+                           "compute streams; each plan's status word read two steps later; CUDA events from "
+                           "before the first plan to the last result on the host"}
 
     others = {}
     cpu = None
