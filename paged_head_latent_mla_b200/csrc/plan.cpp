@@ -347,19 +347,22 @@ mla_status build_layout(const PlanRequest& req, PlanLayout* out) {
     const double avg = (double(total_key_tiles) + kItemCost * tiles.size()) / units;
     // No split can help when the longest tile already fits in the average load of a pair.
     if (req.split_keys == 0 && !tiles.empty() && max_ntiles > 1 && max_ntiles + kItemCost > avg) {
+      // Every chunk size is a candidate (at most ~1000 of them, evenly spaced).
       std::vector<int32_t> cands;
-      for (int32_t dv = 2; dv <= 64; ++dv) cands.push_back((max_ntiles + dv - 1) / dv);
-      for (double f : {1.0, 1.5, 2.0, 3.0, 4.0, 6.0, 8.0}) cands.push_back((int32_t)std::ceil(avg / f));
-      std::sort(cands.begin(), cands.end(), std::greater<int32_t>());
-      cands.erase(std::unique(cands.begin(), cands.end()), cands.end());
-      // Score every candidate by a lower bound on its makespan (the largest of: its
-      // longest item, its average load per pair, and the items some pair must take
-      // times the shortest item; plus the merge pass), then run the full LPT estimate
-      // on the few best.
-      std::vector<std::pair<double, int32_t>> scored;
+      const int32_t stride = std::max<int32_t>(1, (max_ntiles - 2) / 1024);
+      for (int32_t c = 2; c < max_ntiles; c += stride) cands.push_back(c);
+      // Finalists for the full LPT estimate: for each number of waves k (items in k x
+      // pairs), the smallest chunk whose items still fit in k waves (the finest split
+      // with no straggling last wave), and the two candidates with the lowest bound on
+      // the makespan (the largest of: the longest item, the average load per pair, and
+      // the items some pair must take times the shortest item; plus the merge pass).
+      struct Scored {
+        double bound;
+        int32_t chunk;
+        int64_t items;
+      };
+      std::vector<Scored> scored;
       for (int32_t c : cands) {
-        if (c < 2 || c >= max_ntiles) continue;
-        if (!fits(count_for(tiles, n_out, c), req)) continue;
         double longest = 0.0, shortest = std::numeric_limits<double>::infinity(), sum = 0.0, partials = 0.0;
         int64_t items = 0;
         for (const QTile& t : tiles) {
@@ -373,13 +376,25 @@ mla_status build_layout(const PlanRequest& req, PlanLayout* out) {
           if (part) partials += n;
         }
         const double per_unit = double((items + units - 1) / units) * shortest;
-        scored.emplace_back(std::max({longest, sum / units, per_unit}) + kSplitCost * partials / units, c);
+        scored.push_back(Scored{std::max({longest, sum / units, per_unit}) + kSplitCost * partials / units, c, items});
       }
-      std::sort(scored.begin(), scored.end());
+      std::vector<int32_t> finalists;
+      constexpr int64_t kMaxWaves = 6;
+      for (int64_t k = 1; k <= kMaxWaves; ++k) {
+        // cands ascend, items descend: the first candidate within k waves
+        for (const Scored& x : scored)
+          if (x.items <= k * units) {
+            if (finalists.empty() || finalists.back() != x.chunk) finalists.push_back(x.chunk);
+            break;
+          }
+      }
+      std::sort(scored.begin(), scored.end(), [](const Scored& x, const Scored& y) { return x.bound < y.bound; });
+      for (size_t i = 0; i < scored.size() && i < 2; ++i) finalists.push_back(scored[i].chunk);
+      std::sort(finalists.begin(), finalists.end(), std::greater<int32_t>());
+      finalists.erase(std::unique(finalists.begin(), finalists.end()), finalists.end());
       double best = estimate(tiles, 0, units);
-      constexpr size_t kFullEstimates = 4;
-      for (size_t i = 0; i < scored.size() && i < kFullEstimates; ++i) {
-        const int32_t c = scored[i].second;
+      for (int32_t c : finalists) {
+        if (!fits(count_for(tiles, n_out, c), req)) continue;
         // (an estimate that cannot beat best * 0.99 stops early: prefer fewer splits
         // unless clearly better)
         const double e = estimate(tiles, c, units, best * 0.99);
