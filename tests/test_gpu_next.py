@@ -353,3 +353,80 @@ def test_kpe0_is_bitwise_the_rope_kernel_with_zero_q_pe():
     assert torch.equal(o0, o64) and torch.equal(l0, l64)
     p64.destroy()
     p0.destroy()
+
+
+# ------------------------------------------------------------------------- option combinations
+def _replay_steps(steps, H, P, pool, TM, plan_kw, rope=64, append=False, context_only=False):
+    """Capture mla_run (or run-append) once on a graph plan made with `plan_kw`, then for
+    every step: re-plan in place, load the step's inputs, replay, compare with the oracle."""
+    width = 512 + rope
+    d0 = steps[0]
+    plan = M.mla_plan(d0.qo_indptr, d0.kv_indptr, d0.kv_indices, d0.last_page_len, num_heads=H, page_size=P,
+                      num_pages=pool, sm_scale=d0.sm_scale, causal=True, rope_dim=rope,
+                      wait_timeout_ns=TIMEOUT_NS, context_only=context_only, **plan_kw)
+    cache = torch.zeros((pool, P, width), dtype=torch.bfloat16, device=DEV)
+    qn = torch.zeros((TM, H, 512), dtype=torch.bfloat16, device=DEV)
+    qp = torch.zeros((TM, H, 64), dtype=torch.bfloat16, device=DEV) if rope else None
+    kvn = torch.zeros((TM, width), dtype=torch.bfloat16, device=DEV) if append else None
+    out = torch.empty((TM, H, 512), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((TM, H), dtype=torch.float32, device=DEV)
+    s = torch.cuda.Stream()
+    scratch = torch.zeros_like(cache)
+    with torch.cuda.stream(s):
+        M.mla_run(plan, qn, qp, scratch, out=out, lse=lse, kv_new=kvn)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        M.mla_run(plan, qn, qp, cache, out=out, lse=lse, kv_new=kvn)
+    for i, d in enumerate(steps):
+        T = int(d.qo_indptr[-1])
+        c = d.cache[..., :width].contiguous()
+        kv_new = _kv_new(T, 200 + i)[:, :width].contiguous() if append else None
+        with torch.cuda.stream(s):
+            M.mla_plan_update(plan, d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, stream=s.cuda_stream)
+            cache.copy_(c.to(DEV))
+            qn[:T].copy_(d.q_nope.to(DEV))
+            if rope:
+                qp[:T].copy_(d.q_pe.to(DEV))
+            if append:
+                kvn[:T].copy_(kv_new.to(DEV))
+            g.replay()
+        torch.cuda.synchronize()
+        assert M.mla_plan_check(plan) == M.MLA_OK
+        src = O.append_latent(c, kv_new, d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, P) if append else c
+        if append:
+            assert torch.equal(cache.cpu(), torch.from_numpy(src).to(torch.bfloat16))
+        ref_o, ref_l = O.mla_attention(d.q_nope, d.q_pe[..., :rope], src, d.qo_indptr, d.kv_indptr, d.kv_indices,
+                                       d.last_page_len, P, d.sm_scale, causal=True, context_only=context_only)
+        _check(out[:T], lse[:T], ref_o, ref_l)
+    del g
+    info = M.mla_plan_get_info(plan)
+    plan.destroy()
+    return info
+
+
+def test_graph_plan_with_cascade_replays_shared_prefix_steps():
+    pool = 3000
+    steps = [make_custom([4] * 8, [1100 + 40 * i for i in range(8)], 16, 16, shared_group=4, shared_pages=64,
+                         seed=301, pool_pages=pool),
+             make_custom([2] * 6, [1500 + 90 * i for i in range(6)], 16, 16, shared_group=3, shared_pages=80,
+                         seed=302, pool_pages=pool),
+             make_custom([1] * 10, [300 + 77 * i for i in range(10)], 16, 16, seed=303, pool_pages=pool)]
+    _replay_steps(steps, 16, 16, pool, 32, dict(graph_max_batch=12, graph_max_tokens=32, graph_max_page_ids=1500,
+                                                  cascade=True))
+
+
+def test_graph_plan_context_only_replays():
+    pool = 1200
+    steps = [make_custom([3, 1, 5], [3 + 400, 1 + 64, 5 + 900], 128, 64, seed=311, pool_pages=pool),
+             make_custom([2, 2], [2 + 2000, 2 + 10], 128, 64, seed=312, pool_pages=pool)]
+    _replay_steps(steps, 128, 64, pool, 12, dict(graph_max_batch=4, graph_max_tokens=12, graph_max_page_ids=200),
+                  context_only=True)
+
+
+def test_graph_plan_kpe0_with_append_replays():
+    pool = 1200
+    steps = [make_custom([1] * 6, [300 + 500 * i for i in range(6)], 64, 32, seed=321, pool_pages=pool),
+             make_custom([3, 4], [1000, 40], 64, 32, seed=322, pool_pages=pool)]
+    _replay_steps(steps, 64, 32, pool, 8, dict(graph_max_batch=6, graph_max_tokens=8, graph_max_page_ids=400),
+                  rope=0, append=True)

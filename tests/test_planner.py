@@ -275,3 +275,32 @@ def test_graph_plan_bounds_hold_across_steps():
     # the three bounds go together
     with pytest.raises(M.MlaError):
         plan_tables(d0, graph_max_batch=16, graph_max_tokens=64)
+
+
+@pytest.mark.parametrize("H,P,q", [(16, 16, 4), (32, 32, 2), (64, 64, 1)])
+def test_cascade_with_context_only_layout(H, P, q):
+    """Both options together: the shared prefix is cut to the stored context every query
+    of the group sees (c_b = k_b - q_b), and coverage stays exact."""
+    B, group = 8, 4
+    k = [1024 + q + 64 + 29 * i for i in range(B)]
+    d = make_custom([q] * B, k, H, P, shared_group=group, shared_pages=1024 // P, tables_only=True, seed=H)
+    desc = M.mla_plan_describe(plan_tables(d, cascade=True, context_only=True))
+    check_layout(d, desc, context_only=True)
+    assert desc["info"]["num_cascade"] > 0
+
+
+def test_graph_plan_with_cascade_stays_within_capacity():
+    kw = dict(graph_max_batch=16, graph_max_tokens=64, graph_max_page_ids=4096, cascade=True)
+    d0 = make_custom([4] * 16, [1100 + 50 * i for i in range(16)], 16, 16, shared_group=8, shared_pages=64,
+                     tables_only=True, seed=8, pool_pages=6000)
+    p = plan_tables(d0, **kw)
+    cap = M.mla_plan_get_info(p)["work_capacity"]
+    desc = M.mla_plan_describe(p)
+    check_layout(d0, desc)
+    assert desc["info"]["num_cascade"] > 0 and desc["info"]["num_work"] <= cap
+    d1 = make_custom([2] * 12, [2000 + 70 * i for i in range(12)], 16, 16, shared_group=4, shared_pages=100,
+                     tables_only=True, seed=9, pool_pages=6000)
+    M.mla_plan_update(p, d1.qo_indptr, d1.kv_indptr, d1.kv_indices, d1.last_page_len)
+    desc = M.mla_plan_describe(p)
+    check_layout(d1, desc)
+    assert desc["info"]["num_work"] <= cap
