@@ -134,3 +134,34 @@ def test_host_only_plan_cannot_run():
     lib = M.load_library()
     assert lib.mla_run(p.handle, None, None, None, None, None, None) == M.MLA_ERR_INVALID_ARGUMENT
     assert lib.mla_plan_check(p.handle) == M.MLA_OK
+
+
+def test_plain_c_client(tmp_path):
+    """include/mla.h is a C header: a C99 program compiles against it with warnings as
+    errors, links the library, and drives a host-only plan through the ABI."""
+    import shutil
+    import subprocess
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    lib_dir = os.path.dirname(M.LIB_PATH)
+    exe = str(tmp_path / "abi_client")
+    cmd = [cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+           os.path.join(ROOT, "tests", "c", "abi_client.c"), "-L", lib_dir, "-l:libmla_b200.so",
+           "-Wl,-rpath," + lib_dir, "-o", exe]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stdout + r.stderr
+    got = dict((line.split(" ", 1) + [""])[:2] for line in r.stdout.strip().splitlines())
+    assert got["supports"] == "1 1 0"
+    assert got["plan"] == "0 ok"
+    assert got["info"] == "0 batch 2 tokens 4 work 2 merge 0"
+    assert got["kv_len"] == "0 37 150"
+    assert got["update_same"] == "0 1"
+    assert got["update_changed"] == "0 0"
+    assert got["update_bad"] == str(M.MLA_ERR_INVALID_ARGUMENT)
+    assert got["run_host_only"] == str(M.MLA_ERR_INVALID_ARGUMENT)
+    assert got["merge_state_bad"] == str(M.MLA_ERR_INVALID_ARGUMENT)
+    assert "done" in got
