@@ -490,7 +490,9 @@ def measure_next_rows(device, peaks):
       plan) against the same step launched eagerly, device time per step (L2-warm: the
       step reads 215 KB, so this is launch latency);
     * append: mla_append_kv of the mixed chunked-prefill step's 4156 tokens (1152 B read
-      and written per token), L2 flushed before each launch, against HBM bandwidth;
+      and written per token), L2 flushed before each launch, against HBM bandwidth; and
+      mla_run_append against mla_run per step (decode_b64, mixed_prefill), the cost the
+      append adds when the attention is its programmatic dependent;
     * cascade: the speculative shared-prefix rows at 16 heads with and without the cascade;
     * plan reuse: host time of mla_plan_update on an unchanged decode step (skipped
       re-plan) against a changed one and a fresh mla_plan."""
@@ -570,6 +572,45 @@ def measure_next_rows(device, peaks):
     plan.destroy()
     del cache, flush, kv_new
     torch.cuda.empty_cache()
+
+    # --- the append fused ahead of the attention (mla_run_append, the attention launched as
+    # its programmatic dependent) against the attention alone, per step
+    fused = {}
+    for name in ("decode_b64", "mixed_prefill"):
+        d = make_config(name)
+        T = d.total_tokens
+        qn, qp, cache = d.q_nope.to(device), d.q_pe.to(device), d.cache.to(device)
+        kv_new = (torch.randn((T, 576), generator=torch.Generator().manual_seed(6)) * 0.5).to(torch.bfloat16)
+        kv_new = kv_new.to(device)
+        out = torch.empty((T, d.num_heads, 512), dtype=torch.bfloat16, device=device)
+        plan = M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=d.num_heads,
+                          page_size=d.page_size, num_pages=d.num_pages, sm_scale=d.sm_scale, causal=d.causal)
+        # the two variants alternate in short batches, so both see the same clocks (steps of
+        # milliseconds at the power cap drift the SM clock over a long sequence)
+        variants = (("run", {}), ("run_append", {"kv_new": kv_new}))
+        for _ in range(3):
+            for _, kw in variants:
+                M.mla_run(plan, qn, qp, cache, out=out, **kw)
+        torch.cuda.synchronize(device)
+        times = {label: 0.0 for label, _ in variants}
+        batches, per_batch = 4, 5  # short batches keep launches queued back to back
+        for _ in range(batches):
+            for label, kw in variants:
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                for _ in range(per_batch):
+                    M.mla_run(plan, qn, qp, cache, out=out, **kw)
+                b.record()
+                b.synchronize()
+                times[label] += a.elapsed_time(b) / (batches * per_batch) * 1e3
+        if M.mla_plan_check(plan) != 0:
+            raise M.MlaError(M.mla_plan_check(plan), "run_append")
+        plan.destroy()
+        fused[name] = {"tokens": T, "run_us": times["run"], "run_append_us": times["run_append"],
+                       "append_cost_us": times["run_append"] - times["run"]}
+        del qn, qp, cache, kv_new, out
+        torch.cuda.empty_cache()
+    res["run_append_vs_run"] = fused
 
     # --- cascade on/off: the speculative shared-prefix rows with 16 query heads (with 128
     # heads a token fills a query tile by itself and the planner applies no cascade)
