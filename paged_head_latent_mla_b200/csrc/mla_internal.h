@@ -79,6 +79,14 @@ struct PlanLayout {
   int32_t chunk_tiles = 0;  // chosen split size in 64-key tiles (0: no split)
 };
 
+// Planner cost model, in units of one key tile step of a CTA pair: the fixed work of a
+// work item (query load, pipeline fill and drain, epilogue), and the extra of an item
+// whose result is a partial (its write and the merge pass that reads it back).
+constexpr double kItemCost = 3.0;
+constexpr double kSplitCost = 2.0;
+// Split choice: the largest number of waves of SM pairs a split may fill.
+constexpr int kMaxWaves = 6;
+
 // Validate the step's tables and build the work and merge lists (host only).
 mla_status build_layout(const PlanRequest& req, PlanLayout* out);
 

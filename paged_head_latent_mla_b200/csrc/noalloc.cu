@@ -50,6 +50,90 @@ static_assert(kMaxWsRows >= 32 * kTileM, "scratch too small for useful splitting
 WorkItem g_work[kMaxWork];
 MergeItem g_merge[kMaxMerge];
 int32_t g_refs[kMaxWork];
+int32_t g_tile_nt[kMaxWork];    // key tiles of each query tile
+int32_t g_tile_rows[kMaxWork];  // rows of each query tile
+double g_costs[kMaxWork];       // item costs of one split candidate
+constexpr int kMaxUnits = 1024;
+double g_loads[kMaxUnits];
+
+inline int32_t pieces_of(int32_t nt, int32_t chunk) { return (chunk > 0 && nt > chunk) ? (nt + chunk - 1) / chunk : 1; }
+
+// Items, merge records and workspace rows of a split size; false if beyond the scratch.
+bool split_fits(int n_tiles, int32_t chunk, int64_t* items) {
+  int64_t it = 0, merges = 0, rows = 0;
+  for (int i = 0; i < n_tiles; ++i) {
+    const int32_t n = pieces_of(g_tile_nt[i], chunk);
+    it += n;
+    if (n > 1) {
+      ++merges;
+      rows += int64_t(n) * g_tile_rows[i];
+    }
+  }
+  *items = it;
+  return it <= kMaxWork && merges <= kMaxMerge && rows <= kMaxWsRows;
+}
+
+// Longest-first list-scheduling makespan of a split size over `units` SM pairs, the same
+// model as mla_plan's (static buffers only).
+double split_makespan(int n_tiles, int32_t chunk, int units) {
+  int m = 0;
+  int64_t partials = 0;
+  for (int i = 0; i < n_tiles; ++i) {
+    const int32_t nt = g_tile_nt[i], n = pieces_of(nt, chunk);
+    for (int32_t p = 0; p < n; ++p) {
+      const int32_t lo = int32_t(int64_t(nt) * p / n), hi = int32_t(int64_t(nt) * (p + 1) / n);
+      g_costs[m++] = (hi - lo) + kItemCost + (n > 1 ? kSplitCost : 0.0);
+    }
+    if (n > 1) partials += n;
+  }
+  std::sort(g_costs, g_costs + m, [](double a, double b) { return a > b; });
+  for (int u = 0; u < units; ++u) g_loads[u] = 0.0;
+  double worst = 0.0;
+  for (int i = 0; i < m; ++i) {
+    int best = 0;
+    for (int u = 1; u < units; ++u)
+      if (g_loads[u] < g_loads[best]) best = u;
+    g_loads[best] += g_costs[i];
+    worst = std::max(worst, g_loads[best]);
+  }
+  return worst + kSplitCost * double(partials) / units;
+}
+
+// The split size: no split when no query tile exceeds the average load of a pair;
+// otherwise, for each wave count k, the finest split whose items fit in k waves of the
+// pairs, scored by the makespan model (a split must be 1% better than the one before).
+int32_t choose_chunk(int n_tiles, int64_t total_tiles, int units) {
+  int32_t max_nt = 0;
+  for (int i = 0; i < n_tiles; ++i) max_nt = std::max(max_nt, g_tile_nt[i]);
+  const double avg = (double(total_tiles) + kItemCost * n_tiles) / units;
+  if (n_tiles == 0 || max_nt <= 1 || max_nt + kItemCost <= avg) return 0;
+  int32_t chunk = 0;
+  double best = split_makespan(n_tiles, 0, units);
+  int32_t last_tried = -1;
+  for (int k = 1; k <= kMaxWaves; ++k) {
+    // items(c) does not increase with c: bisect for the smallest c within k waves
+    int32_t lo = 2, hi = max_nt - 1, found = -1;
+    while (lo <= hi) {
+      const int32_t mid = lo + (hi - lo) / 2;
+      int64_t items = 0;
+      const bool ok = split_fits(n_tiles, mid, &items);
+      if (items <= int64_t(k) * units) {
+        if (ok) found = mid;
+        hi = mid - 1;
+      } else {
+        lo = mid + 1;
+      }
+    }
+    if (found < 0 || found == last_tried) continue;
+    last_tried = found;
+    const double e = split_makespan(n_tiles, found, units);
+    if (e < best * 0.99) {
+      best = e;
+      chunk = found;
+    }
+  }
+  return chunk;
+}
 
 struct DeviceScratch {
   unsigned char* ptr = nullptr;
@@ -59,9 +143,9 @@ constexpr int kMaxDevices = 64;
 DeviceScratch g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
 
-// Validate the tables and cut the work into g_work / g_merge without allocating.
-// Long key ranges are split into chunks of about (total tiles / SM pairs) tiles while
-// workspace rows remain in the scratch array; the rest run unsplit.
+// Validate the tables and cut the work into g_work / g_merge without allocating.  The
+// split size follows mla_plan's rule (whole waves of SM pairs, the same cost model), kept
+// within the scratch array; a tile whose pieces would not fit the rest runs unsplit.
 mla_status plan_fixed(const mla_dims& d, int32_t batch, const int32_t* qo, const int32_t* kvp,
                       const int32_t* kvi, const int32_t* last, bool causal, int num_sms, int* n_work,
                       int* n_merge, int* n_refs, int* n_ws_rows, int32_t* total_tokens) {
@@ -93,13 +177,15 @@ mla_status plan_fixed(const mla_dims& d, int32_t batch, const int32_t* qo, const
       const int32_t ntok = std::min(tok_per_tile, q_b - tok0);
       const int64_t diag = causal ? k - q_b + tok0 : k;
       const int64_t hi = std::max<int64_t>(0, std::min<int64_t>(causal ? diag + ntok : k, k));
-      total_tiles += (hi + kTileN - 1) / kTileN;
+      if (n_tiles >= kMaxWork) return MLA_ERR_INVALID_ARGUMENT;  // beyond the fixed scratch
+      g_tile_nt[n_tiles] = static_cast<int32_t>((hi + kTileN - 1) / kTileN);
+      g_tile_rows[n_tiles] = ntok * H;
+      total_tiles += g_tile_nt[n_tiles];
       ++n_tiles;
     }
   }
-  if (n_tiles > kMaxWork) return MLA_ERR_INVALID_ARGUMENT;  // beyond the fixed scratch
-  const int units = std::max(1, num_sms / 2);
-  const int64_t chunk = std::max<int64_t>(8, (total_tiles + units - 1) / units);
+  const int units = std::min(kMaxUnits, std::max(1, num_sms / 2));
+  const int32_t chunk = choose_chunk(static_cast<int>(n_tiles), total_tiles, units);
   // pass 2: emit (every tile still to come keeps at least one work slot)
   int nw = 0, nm = 0, nr = 0, rows_used = 0;
   int64_t tiles_left = n_tiles;
@@ -114,7 +200,7 @@ mla_status plan_fixed(const mla_dims& d, int32_t batch, const int32_t* qo, const
       const int32_t vis_hi = static_cast<int32_t>(hi64);
       const int32_t nt = (vis_hi + kTileN - 1) / kTileN;
       const int32_t q_row0 = (qo[b] + tok0) * H;
-      int32_t pieces = nt > chunk ? static_cast<int32_t>((nt + chunk - 1) / chunk) : 1;
+      int32_t pieces = pieces_of(nt, chunk);
       --tiles_left;
       if (pieces > 1 && (rows_used + pieces * ntok * H > kMaxWsRows || nm >= kMaxMerge ||
                          nw + pieces + tiles_left > kMaxWork))

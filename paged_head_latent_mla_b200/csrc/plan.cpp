@@ -56,12 +56,6 @@ struct QTile {
   int32_t first_out, n_out;  // output tiles covered (cascade tiles)
 };
 
-// Cost, in units of one key tile step, of the fixed work of one item: query load,
-// pipeline fill/drain and epilogue.  Split items also write a partial that the merge
-// kernel reads back.
-constexpr double kItemCost = 3.0;
-constexpr double kSplitCost = 2.0;
-
 // Longest-processing-time-first makespan of `costs` over `units` identical units.  Stops
 // early (returning a value >= `give_up`) once the makespan cannot end below `give_up`.
 double lpt_makespan(std::vector<double>& costs, int units, double give_up) {
@@ -379,7 +373,6 @@ mla_status build_layout(const PlanRequest& req, PlanLayout* out) {
         scored.push_back(Scored{std::max({longest, sum / units, per_unit}) + kSplitCost * partials / units, c, items});
       }
       std::vector<int32_t> finalists;
-      constexpr int64_t kMaxWaves = 6;
       for (int64_t k = 1; k <= kMaxWaves; ++k) {
         // cands ascend, items descend: the first candidate within k waves
         for (const Scored& x : scored)
