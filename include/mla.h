@@ -278,9 +278,10 @@ mla_status mla_plan_kernel_times(mla_plan_t plan, int32_t capacity, float* attn_
  * not (no cudaMalloc, cudaFree or pinned allocation, and no heap use while planning).
  *
  * Arguments are those of mla_plan (host tables, copied during the call) followed by
- * those of mla_run (device tensors, same layouts and alignment rules).  Planning uses a
- * fixed split rule instead of mla_plan's balancing search, so the split points may
- * differ from mla_run's; results agree within floating-point tolerance.
+ * those of mla_run (device tensors, same layouts and alignment rules).  Planning follows
+ * mla_plan's split rule within the fixed scratch below (long rows beyond its room run
+ * unsplit), so the split points may differ from mla_run's; results agree within
+ * floating-point tolerance.  No graph, context-only or cascade options.
  *
  * All device scratch (status word, work list, page-table copy, split-KV partials) lives
  * in one 16 MiB array compiled into the library; every GPU that loads the library holds
