@@ -86,6 +86,9 @@ constexpr double kItemCost = 3.0;
 constexpr double kSplitCost = 2.0;
 // Split choice: the largest number of waves of SM pairs a split may fill.
 constexpr int kMaxWaves = 6;
+// When every item has an SM pair to itself, a split step lasts its longest item plus the
+// merge launch that follows (about one key tile step).
+constexpr double kMergeLatency = 1.0;
 
 // Validate the step's tables and build the work and merge lists (host only).
 mla_status build_layout(const PlanRequest& req, PlanLayout* out);

@@ -398,6 +398,37 @@ mla_status build_layout(const PlanRequest& req, PlanLayout* out) {
       }
     }
   }
+  // Latency regime: when the items fit in one wave, every item runs on its own pair and
+  // the step lasts as long as its longest item (plus a merge launch if anything is
+  // split), so split the longest tiles further, down to single key tiles, while the
+  // items still fit one wave (a tiny decode step: 14.8 us instead of 16.8 us).
+  if (req.split_keys == 0 && !tiles.empty() && max_ntiles > 1) {
+    auto latency = [&](int32_t c, int64_t* items) {
+      double longest = 0.0;
+      int64_t it = 0, partials = 0;
+      for (const QTile& t : tiles) {
+        const int32_t n = c > 0 ? pieces_for(t.ntiles, c) : 1;
+        it += n;
+        if (n > 1 || t.must_merge) partials += n;
+        longest = std::max(longest, double((t.ntiles + n - 1) / n) + kItemCost);
+      }
+      *items = it;
+      return longest + (partials > 0 ? kMergeLatency : 0.0);
+    };
+    int64_t items = 0;
+    double best_lat = latency(chunk, &items);
+    if (items <= units) {
+      for (int32_t c = std::max<int32_t>(1, chunk > 0 ? chunk - 1 : max_ntiles - 1); c >= 1; --c) {
+        int64_t it = 0;
+        const double l = latency(c, &it);
+        if (it > units) break;  // finer splits only add items
+        if (l < best_lat * 0.99 && fits(count_for(tiles, n_out, c), req)) {
+          best_lat = l;
+          chunk = c;
+        }
+      }
+    }
+  }
   out->chunk_tiles = chunk;
 
   // --- emit items and the merge references of every output tile

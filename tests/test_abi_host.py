@@ -157,7 +157,7 @@ def test_plain_c_client(tmp_path):
     got = dict((line.split(" ", 1) + [""])[:2] for line in r.stdout.strip().splitlines())
     assert got["supports"] == "1 1 0"
     assert got["plan"] == "0 ok"
-    assert got["info"] == "0 batch 2 tokens 4 work 2 merge 0"
+    assert got["info"] == "0 batch 2 tokens 4 work 4 merge 1"  # the 3-tile row split for latency
     assert got["kv_len"] == "0 37 150"
     assert got["update_same"] == "0 1"
     assert got["update_changed"] == "0 0"

@@ -69,8 +69,12 @@ def compare(d, out, lse, tokens=None):
 def test_tiny_decode_config():
     d = make_config("tiny_decode")
     out, lse, info, _ = gpu_run(d)
-    assert info["num_work"] == 2
+    # the 3-tile row is cut into single tiles for latency (4 items, one merge)
+    assert info["num_work"] == 4 and info["num_merge"] == 1
     compare(d, out, lse)
+    out1, lse1, info1, _ = gpu_run(d, split_keys=-1)  # and unsplit
+    assert info1["num_work"] == 2
+    compare(d, out1, lse1)
 
 
 @pytest.mark.parametrize("H", [16, 32, 64, 128])

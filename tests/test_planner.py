@@ -178,10 +178,19 @@ def test_auto_split_balances_long_decode():
     assert max(lens) / T <= 2 * (sum(lens) / T) / 74 + 8
 
 
-def test_no_split_for_small_decode():
+def test_small_decode_splits_for_latency_within_one_wave():
+    """With fewer items than SM pairs the step lasts as long as its longest item: the
+    tiny decode step's 3-tile row is cut into single tiles (4 items, one merge), while a
+    step whose single-tile split would exceed one wave keeps its throughput split."""
     d = make_config("tiny_decode", tables_only=True)
     desc = M.mla_plan_describe(plan_tables(d))
-    assert desc["info"]["num_merge"] == 0 and desc["info"]["num_work"] == 2
+    assert desc["info"]["num_work"] == 4 and desc["info"]["num_merge"] == 1
+    assert max(w[5] - w[4] for w in desc["work"]) <= M.MLA_KEY_TILE
+    check_layout(d, desc)
+    d8 = make_custom([1] * 8, [300 + 97 * i for i in range(8)], 128, 64, seed=5, tables_only=True)
+    desc = M.mla_plan_describe(plan_tables(d8))
+    assert desc["info"]["num_work"] <= 74
+    check_layout(d8, desc)
 
 
 @pytest.mark.parametrize("H,P,q", [(128, 64, 4), (16, 16, 4), (16, 16, 3), (32, 32, 1), (64, 128, 2), (64, 64, 1)])
