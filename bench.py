@@ -340,6 +340,7 @@ def time_workload(d, device, steps, warmup, dist=None, soak_s=0.0, sampler=None,
         if st != 0:
             raise M.MlaError(st, "timed steps")
     res = {"ms_total": ms, "ms_per_step": ms / steps, "attn_ms": float(attn_ms.mean()),
+           "attn_ms_median": float(statistics.median(attn_ms.tolist())), "attn_ms_min": float(attn_ms.min()),
            "merge_ms": float(merge_ms.mean()), "info": info, "n_copies": n_copies, "clocks": clocks,
            "launches": steps * (1 + (1 if info["num_merge"] > 0 else 0))}
     plan.destroy()
@@ -451,6 +452,8 @@ def summarise(d, res, peaks):
     return {
         "us_per_step": res["ms_per_step"] * 1e3,
         "attn_kernel_us": res["attn_ms"] * 1e3,
+        "attn_kernel_us_median": res["attn_ms_median"] * 1e3,
+        "attn_kernel_us_min": res["attn_ms_min"] * 1e3,
         "merge_kernel_us": res["merge_ms"] * 1e3,
         "kv_gbs": w["kv_bytes"] / s / 1e9,
         "tflops": w["flops"] / s / 1e12,
@@ -757,6 +760,8 @@ def run_native(args):
         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
         "algorithmic_bytes_per_launch": w["kv_bytes"],
         "kernel_us": res["attn_ms"] * 1e3,
+        "kernel_us_median": res["attn_ms_median"] * 1e3,
+        "kernel_us_min": res["attn_ms_min"] * 1e3,
         "tensor_achieved_tflops": w["flops"] / attn_s / 1e12,
         "tensor_frac": w["flops"] / attn_s / 1e12 / peaks["bf16_tflops"],
         "note": "decode at H=128 does 242 flop per KV byte, just under the ridge; both fractions are reported",
