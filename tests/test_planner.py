@@ -313,3 +313,79 @@ def test_graph_plan_with_cascade_stays_within_capacity():
     desc = M.mla_plan_describe(p)
     check_layout(d1, desc)
     assert desc["info"]["num_work"] <= cap
+
+
+# ----------------------------------------------------------------------------- properties
+from hypothesis import HealthCheck, given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+
+@st.composite
+def _step(draw):
+    H = draw(st.sampled_from([16, 32, 64, 128]))
+    P = draw(st.sampled_from([16, 32, 64, 128]))
+    B = draw(st.integers(0, 10))
+    q = [draw(st.integers(0, 24)) for _ in range(B)]
+    k = [draw(st.integers(0, 900)) for _ in range(B)]
+    causal = draw(st.booleans())
+    context_only = draw(st.booleans())
+    if context_only:
+        k = [max(ki, qi) for ki, qi in zip(k, q)]
+    group = draw(st.sampled_from([0, 2, 3]))
+    shared = 0
+    if group and B and min(k) >= 2 * P:
+        shared = draw(st.integers(1, min(k) // P))
+    split = draw(st.sampled_from([0, 0, -1, 64, 192, 512]))
+    cascade = draw(st.booleans())
+    return dict(H=H, P=P, q=q, k=k, causal=causal, context_only=context_only, group=group, shared=shared,
+                split=split, cascade=cascade)
+
+
+@settings(max_examples=150, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(_step())
+def test_random_steps_keep_exact_bookkeeping(c):
+    """Any valid step, with any mix of options, plans to work items that cover every
+    visible key of every query exactly once, with merge references that reach every
+    partial once and a kernel visibility rule that matches the oracle's."""
+    d = make_custom(c["q"], c["k"], c["H"], c["P"], causal=c["causal"], tables_only=True, extra_pool_pages=2,
+                    shared_group=c["group"] if c["shared"] else 0, shared_pages=c["shared"])
+    p = plan_tables(d, split_keys=c["split"], cascade=c["cascade"], context_only=c["context_only"])
+    desc = M.mla_plan_describe(p)
+    check_layout(d, desc, context_only=c["context_only"])
+    if c["split"] > 0:
+        assert all(w[5] - w[4] <= c["split"] for w in desc["work"])
+
+
+@settings(max_examples=60, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(st.lists(st.tuples(st.lists(st.integers(0, 6), min_size=1, max_size=8),
+                          st.lists(st.integers(0, 3000), min_size=8, max_size=8)), min_size=2, max_size=5),
+       st.sampled_from([16, 64, 128]), st.booleans())
+def test_graph_plan_sequences_keep_bookkeeping_and_capacity(steps, H, cascade):
+    """A graph plan re-planned through a random sequence of steps of its bucket keeps
+    exact bookkeeping and never exceeds the launch capacity it was made with; a step
+    outside the bucket is rejected without changing the plan."""
+    pool = 500
+    first = None
+    plan = None
+    cap = None
+    for q, k in steps:
+        k = [max(ki, 1) for ki in k[: len(q)]]
+        d = make_custom(q, k, H, 64, tables_only=True, pool_pages=pool, seed=len(q) + sum(k) % 97)
+        if int(d.kv_indptr[-1]) > 400 or sum(q) > 48:
+            continue
+        if plan is None:
+            plan = plan_tables(d, graph_max_batch=8, graph_max_tokens=48, graph_max_page_ids=400, cascade=cascade)
+            cap = M.mla_plan_get_info(plan)["work_capacity"]
+            first = d
+        else:
+            M.mla_plan_update(plan, d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len)
+        desc = M.mla_plan_describe(plan)
+        check_layout(d, desc)
+        assert desc["info"]["num_work"] <= cap and desc["info"]["work_capacity"] == cap
+    if plan is not None:
+        before = M.mla_plan_describe(plan)["work"].copy()
+        big = make_custom([1] * 9, [64] * 9, H, 64, tables_only=True, pool_pages=pool)  # 9 rows > 8
+        with pytest.raises(M.MlaError):
+            M.mla_plan_update(plan, big.qo_indptr, big.kv_indptr, big.kv_indices, big.last_page_len)
+        assert np.array_equal(M.mla_plan_describe(plan)["work"], before)
+        assert first is not None
