@@ -430,3 +430,44 @@ def test_graph_plan_kpe0_with_append_replays():
              make_custom([3, 4], [1000, 40], 64, 32, seed=322, pool_pages=pool)]
     _replay_steps(steps, 64, 32, pool, 8, dict(graph_max_batch=6, graph_max_tokens=8, graph_max_page_ids=400),
                   rope=0, append=True)
+
+
+# ------------------------------------------------------------------------- random steps
+from hypothesis import HealthCheck, given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+
+@st.composite
+def _gpu_step(draw):
+    H = draw(st.sampled_from([16, 64, 128]))
+    P = draw(st.sampled_from([16, 64]))
+    B = draw(st.integers(1, 5))
+    q = [draw(st.integers(0, 9)) for _ in range(B)]
+    k = [draw(st.integers(0, 700)) for _ in range(B)]
+    context_only = draw(st.booleans())
+    if context_only:
+        k = [max(ki, qi) for ki, qi in zip(k, q)]
+    return dict(H=H, P=P, q=q, k=k, causal=draw(st.booleans()), context_only=context_only,
+                cascade=draw(st.booleans()), split=draw(st.sampled_from([0, -1, 128])),
+                rope=draw(st.sampled_from([64, 0])), seed=draw(st.integers(0, 1000)))
+
+
+@settings(max_examples=12, deadline=None, derandomize=True, suppress_health_check=[HealthCheck.too_slow])
+@given(_gpu_step())
+def test_random_steps_match_oracle(c):
+    """Small random steps with a random mix of options, element by element against the
+    oracle (a fixed, derandomized sample of cases)."""
+    d = make_custom(c["q"], c["k"], c["H"], c["P"], causal=c["causal"], seed=c["seed"], extra_pool_pages=2)
+    R = c["rope"]
+    cache = d.cache[..., :512 + R].contiguous()
+    plan = M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=c["H"], page_size=c["P"],
+                      num_pages=d.num_pages, sm_scale=d.sm_scale, causal=c["causal"], rope_dim=R,
+                      split_keys=c["split"], cascade=c["cascade"], context_only=c["context_only"],
+                      wait_timeout_ns=TIMEOUT_NS)
+    out, lse = M.mla_run(plan, d.q_nope.to(DEV), d.q_pe.to(DEV) if R else None, cache.to(DEV), return_lse=True)
+    assert M.mla_plan_check(plan) == M.MLA_OK
+    plan.destroy()
+    ref_o, ref_l = O.mla_attention(d.q_nope, d.q_pe[..., :R], cache, d.qo_indptr, d.kv_indptr, d.kv_indices,
+                                   d.last_page_len, c["P"], d.sm_scale, causal=c["causal"],
+                                   context_only=c["context_only"])
+    _check(out, lse, ref_o, ref_l)
