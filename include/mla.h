@@ -217,7 +217,9 @@ mla_status mla_plan_describe(mla_plan_t plan, int32_t* kv_len, int32_t* work, in
  * plan is unchanged.  Other plans may grow their buffers (waiting for their last run
  * first when they do).  The host staging is double-buffered: the call waits only for
  * the upload of two updates ago, so the host may run one step ahead of the GPU
- * (FlashInferMLAManager.force_double_buffer describes the race this avoids).
+ * (FlashInferMLAManager.force_double_buffer describes the race this avoids).  It must
+ * not be called while `stream` is being captured into a graph (the upload belongs to
+ * the moment of re-planning, not to every replay): INVALID_ARGUMENT.
  * Errors: INVALID_ARGUMENT, OUT_OF_MEMORY, CUDA; on error the plan still describes and
  * runs its previous step. */
 mla_status mla_plan_update(mla_plan_t plan, int32_t batch, const int32_t* qo_indptr, const int32_t* kv_indptr,
