@@ -19,13 +19,18 @@
 //    288 of the 576 contraction columns.  Each CTA TMA-gathers only its columns of
 //    every key, so every cache byte crosses HBM once.
 //  * Per 64-key tile: each CTA computes a partial S = Q_half . K_half^T (tcgen05,
-//    M=128, N=64, K=288) into TMEM; the softmax warps push their partial to the peer
-//    over DSMEM, add the peer's partial (fp32 addition commutes, so both CTAs hold
-//    bit-identical S), apply mask and online softmax (log2 domain, lazy rescale), and
-//    store P as bf16 into TMEM.  Then O_half += P . V_half (tcgen05, A = P from TMEM,
-//    B = the ckv columns of the same shared-memory tile read MN-major, N = 256).
-//  * Roles: warp 0 issues TMA, warp 1 issues MMAs (one thread) and zeroes key rows
-//    past the row's end, warps 2..5 run softmax, exchange and epilogue.
+//    M=128, N=64, K=288) into TMEM; the exchange warps push it to the peer over DSMEM
+//    (st.async completing on the peer's mbarrier); the softmax warps add the peer's
+//    partial (fp32 addition commutes, so both CTAs hold bit-identical S), apply mask
+//    and online softmax (log2 domain, lazy rescale), and store P as bf16 into TMEM.
+//    Then O_half += P . V_half (tcgen05, A = P from TMEM, B = the ckv columns of the
+//    same shared-memory tile read MN-major, N = 256).
+//  * Roles (11 warps): warps 0..3 softmax and epilogue, 4..7 exchange (one per TMEM
+//    lane quarter in each group), 8 TMA producer, 9 QK issuer (one thread; also TMEM
+//    allocation and zeroing of key rows past the row's end), 10 PV issuer.
+//  * An empty work item (an unused launch slot of a graph plan) returns at once; the
+//    producer waits for a preceding cache append (programmatic dependent launch)
+//    before its first key load; the kpe width is a run-time parameter (64 or 0).
 //  * Every wait is bounded; on timeout the kernel records MLA_ERR_DEVICE_TIMEOUT in
 //    the plan's status word and every role unwinds.
 #include <cuda.h>
