@@ -230,6 +230,30 @@ def check_lse_merge(oracle):
         np.testing.assert_allclose(ml3, full_lse[0], rtol=1e-12, atol=1e-13)
 
 
+def check_merge_closed_forms(oracle):
+    """Closed forms of the two-state merge: an empty state (lse = -inf) is the identity;
+    a state merged with itself keeps its output and gains ln 2; two equal-lse states
+    average their outputs; a state whose lse is far below the other's leaves it unchanged
+    to rounding."""
+    rng = np.random.default_rng(41)
+    o = rng.normal(size=(5, D_C))
+    l = rng.normal(size=5) * 3
+    e_o, e_l = np.zeros_like(o), np.full(5, -np.inf)
+    mo, ml = oracle.merge_states(o, l, e_o, e_l)
+    assert np.array_equal(mo, o) and np.array_equal(ml, l)
+    mo, ml = oracle.merge_states(e_o, e_l, e_o, e_l)
+    assert np.all(mo == 0) and np.all(np.isneginf(ml))
+    mo, ml = oracle.merge_states(o, l, o, l)
+    np.testing.assert_allclose(mo, o, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(ml, l + math.log(2.0), rtol=0, atol=1e-14)
+    o2 = rng.normal(size=(5, D_C))
+    mo, ml = oracle.merge_states(o, l, o2, l)
+    np.testing.assert_allclose(mo, (o + o2) / 2, rtol=0, atol=1e-14)
+    mo, ml = oracle.merge_states(o, l, o2, l - 800.0)
+    np.testing.assert_allclose(mo, o, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(ml, l, rtol=0, atol=1e-14)
+
+
 def check_empty_and_overhang(oracle):
     # k = 0 row, and a causal row with more queries than keys
     d = _paged([2, 5], [0, 3], 2, 4, seed=4)
@@ -374,6 +398,7 @@ ALL_CHECKS = [
     check_page_permutation,
     check_causal_noop_single_query,
     check_lse_merge,
+    check_merge_closed_forms,
     check_empty_and_overhang,
     check_kv_lengths,
     check_append_slots,
