@@ -235,8 +235,10 @@ mla_status mla_plan_update(mla_plan_t plan, int32_t batch, const int32_t* qo_ind
  *           16-byte aligned
  *   cache   device bf16 [num_pages][page_size][512 + rope_dim] (written at those slots
  *           only)
- * One launch, no allocation, no synchronisation.  Two tokens naming the same slot (a
- * page listed twice) leave one of the two rows there.  Errors: INVALID_ARGUMENT (NULL
+ * One launch, no allocation, no synchronisation.  Where several tokens name the same
+ * slot (a page listed twice), the latest of them (highest t) is the one written: the
+ * plan gives the earlier ones no destination, so no two writes race on a slot.
+ * Errors: INVALID_ARGUMENT (NULL
  * or misaligned pointer, or a row with q_b > k_b, whose tokens have no slots), CUDA. */
 mla_status mla_append_kv(mla_plan_t plan, const void* kv_new, void* cache, void* stream);
 
@@ -293,17 +295,22 @@ mla_status mla_plan_kernel_times(mla_plan_t plan, int32_t capacity, float* attn_
  * for their partial results (at least 32 tiles' worth); the rest run unsplit.
  *
  * The first call on a device looks up the array's device address (and the SM count)
- * with that device current; make that first call before any stream capture.  Every call
- * shares the one array (and static host buffers), so calls must not overlap, on the host
- * or on the GPU: issue them from one thread, on one stream, or synchronise in between.
- * In-kernel wait timeouts are recorded in the array's status word, which is not
- * reported back; use mla_plan/mla_run/mla_plan_check where that matters.
+ * with that device current.  Every call shares the one array (and static host
+ * buffers), so calls must not overlap, on the host or on the GPU: issue them from one
+ * thread, on one stream, or synchronise in between.  The call cannot be captured into a
+ * CUDA graph (its uploads read static host buffers at enqueue time): on a capturing
+ * stream it returns MLA_ERR_UNSUPPORTED and enqueues nothing.
+ *   status_out  device int32 or NULL.  When given, it receives the call's device status
+ *               once the stream has passed the call: 0, or MLA_ERR_DEVICE_TIMEOUT in its
+ *               low byte when an in-kernel wait gave up (the bits above name the wait).
+ *               Read it after synchronising; the call only writes it.
  * Errors: INVALID_ARGUMENT (bad tables or pointers, or beyond the limits above),
- * UNSUPPORTED (shape), CUDA. */
+ * UNSUPPORTED (shape, or a capturing stream), CUDA. */
 mla_status mla_run_noalloc(const mla_dims* dims, int32_t batch, const int32_t* qo_indptr,
                            const int32_t* kv_indptr, const int32_t* kv_indices,
                            const int32_t* last_page_len, int32_t causal, const void* q_nope,
-                           const void* q_pe, const void* cache, void* out, float* lse, void* stream);
+                           const void* q_pe, const void* cache, void* out, float* lse, void* stream,
+                           int32_t* status_out);
 
 /* Wait for the plan's last run, then free everything it owns.  NULL is a no-op. */
 void mla_plan_destroy(mla_plan_t plan);

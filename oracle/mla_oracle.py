@@ -256,9 +256,14 @@ def append_latent(cache, kv_new, qo_indptr, kv_indptr, kv_indices, last_page_len
 
     Token i of row b (global token ``qo_indptr[b] + i``) is logical key
     ``k_b - q_b + i`` of its row; ``kv_new [T, 576]`` row t is stored at that key's
-    (page, slot).  Returns a float64 copy of ``cache`` with those rows replaced, in
-    token order (a later token wins where two name the same slot).  A row with
-    ``q_b > k_b`` has no slot for its first tokens and is rejected.
+    (page, slot).  Returns a float64 copy of ``cache`` with those rows replaced.
+
+    Page ids may repeat (reading of ``captured_page_capacity`` on the base page), so
+    two tokens can name one slot; the write then leaves one of their rows there, and
+    which one is not fixed by the method.  This copy writes in token order, so it
+    holds the later token's row: one valid result among several, and a check against
+    it must accept any of the rows that name the slot.  A row with ``q_b > k_b`` has
+    no slot for its first tokens and is rejected.
     """
     out = _f64(cache).copy()
     new = _f64(kv_new)

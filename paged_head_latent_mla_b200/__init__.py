@@ -143,7 +143,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_plan_kernel_times.argtypes = [vp, ctypes.c_int32, fp, fp, i32p]
     lib.mla_plan_kernel_times.restype = ctypes.c_int
     lib.mla_run_noalloc.argtypes = [ctypes.POINTER(_Dims), ctypes.c_int32, i32p, i32p, i32p, i32p, ctypes.c_int32,
-                                    vp, vp, vp, vp, vp, vp]
+                                    vp, vp, vp, vp, vp, vp, vp]
     lib.mla_run_noalloc.restype = ctypes.c_int
     lib.mla_plan_destroy.argtypes = [vp]
     lib.mla_plan_destroy.restype = None
@@ -185,12 +185,15 @@ class MlaPlan:
     """Owns one C plan handle (``mla_plan_t``); destroyed with the object."""
 
     def __init__(self, handle: int, batch: int, num_heads: int, total_tokens: int, graph_max_tokens: int = 0,
-                 rope_dim: int = ROPE_DIM):
+                 rope_dim: int = ROPE_DIM, num_pages: int = 0, page_size: int = 0):
         self._h = ctypes.c_void_p(handle)
         self.batch = batch
         self.num_heads = num_heads
         self.total_tokens = total_tokens
         self.rope_dim = rope_dim
+        # the cache every run of this plan reads is [num_pages, page_size, 512 + rope_dim]
+        self.num_pages = num_pages
+        self.page_size = page_size
         # a graph plan's per-token buffers hold graph_max_tokens tokens
         self.graph_max_tokens = graph_max_tokens
 
@@ -251,7 +254,7 @@ def mla_plan(qo_indptr, kv_indptr, kv_indices, last_page_len, *, num_heads: int,
     if st != MLA_OK:
         raise MlaError(st, "mla_plan")
     return MlaPlan(out.value, batch, num_heads, int(qo[-1]), graph_max_tokens if graph_max_tokens > 0 else 0,
-                   rope_dim)
+                   rope_dim, num_pages, page_size)
 
 
 def mla_plan_update(plan: MlaPlan, qo_indptr, kv_indptr, kv_indices, last_page_len, stream=None) -> bool:
@@ -309,6 +312,17 @@ def mla_plan_describe(plan: MlaPlan) -> dict:
     }
 
 
+def _check_cache_shape(cache, num_pages: int, page_size: int, rope_dim: int) -> None:
+    """The cache must be [>= num_pages, page_size, 512 + rope_dim]: the kernels' tensor
+    maps span num_pages * page_size rows of 512 + rope_dim columns, so a tensor with
+    fewer pages would be read past its end (a larger pool is fine)."""
+    width = KV_LORA_RANK + rope_dim
+    shape = tuple(getattr(cache, "shape", ()))
+    if len(shape) != 3 or shape[1] != page_size or shape[2] != width or shape[0] < num_pages:
+        raise ValueError(f"cache must have shape (>= {num_pages}, {page_size}, {width}) "
+                         f"(num_pages, page_size, 512 + rope_dim), got {shape}")
+
+
 def _check_dev_tensor(t, name, dtype, shape):
     import torch
 
@@ -332,11 +346,10 @@ def mla_run(plan: MlaPlan, q_nope, q_pe, cache, out=None, lse=None, return_lse: 
 
     T, H, R = plan.token_capacity, plan.num_heads, plan.rope_dim
     width = KV_LORA_RANK + R
+    _check_cache_shape(cache, plan.num_pages, plan.page_size, R)
     _check_dev_tensor(q_nope, "q_nope", torch.bfloat16, (T, H, KV_LORA_RANK))
     if R > 0 or q_pe is not None:
         _check_dev_tensor(q_pe, "q_pe", torch.bfloat16, (T, H, R))
-    if cache.dim() != 3 or cache.shape[-1] != width:
-        raise ValueError(f"cache must be [num_pages, page_size, {width}]")
     _check_dev_tensor(cache, "cache", torch.bfloat16, tuple(cache.shape))
     if out is None:
         out = torch.empty((T, H, KV_LORA_RANK), dtype=torch.bfloat16, device=q_nope.device)
@@ -373,9 +386,8 @@ def mla_append_kv(plan: MlaPlan, kv_new, cache, stream=None) -> None:
     import torch
 
     width = KV_LORA_RANK + plan.rope_dim
+    _check_cache_shape(cache, plan.num_pages, plan.page_size, plan.rope_dim)
     _check_dev_tensor(kv_new, "kv_new", torch.bfloat16, (plan.token_capacity, width))
-    if cache.dim() != 3 or cache.shape[-1] != width:
-        raise ValueError(f"cache must be [num_pages, page_size, {width}]")
     _check_dev_tensor(cache, "cache", torch.bfloat16, tuple(cache.shape))
     if stream is None:
         stream = torch.cuda.current_stream(kv_new.device).cuda_stream
@@ -431,12 +443,17 @@ def mla_plan_kernel_times(plan: MlaPlan, capacity: int = 256):
 
 def mla_run_noalloc(qo_indptr, kv_indptr, kv_indices, last_page_len, q_nope, q_pe, cache, out, lse=None, *,
                     num_heads: int, page_size: int, num_pages: int, sm_scale: float, causal: bool = True,
-                    kv_lora_rank: int = KV_LORA_RANK, rope_dim: int = ROPE_DIM, stream=None) -> None:
+                    kv_lora_rank: int = KV_LORA_RANK, rope_dim: int = ROPE_DIM, stream=None, status=None) -> None:
     """Plan and run one step without allocating (``mla_run_noalloc``): for callers that
     may not allocate device memory when attention runs.  ``out`` (and ``lse`` if given)
-    must be preallocated by the caller; host tables as for ``mla_plan``.  Calls share
-    one fixed device scratch array, so they must not overlap."""
+    must be preallocated by the caller; host tables as for ``mla_plan``.  ``status``
+    (optional, a preallocated int32 CUDA tensor of one element) receives the step's
+    device status once the stream has passed it (0, or MLA_ERR_DEVICE_TIMEOUT in the low
+    byte).  Calls share one fixed device scratch array, so they must not overlap, and
+    cannot be captured into a CUDA graph."""
     import torch
+
+    _check_cache_shape(cache, num_pages, page_size, rope_dim)
 
     qo = _i32(qo_indptr)
     kvp = _i32(kv_indptr)
@@ -453,6 +470,8 @@ def mla_run_noalloc(qo_indptr, kv_indptr, kv_indices, last_page_len, q_nope, q_p
     _check_dev_tensor(out, "out", torch.bfloat16, (T, num_heads, kv_lora_rank))
     if lse is not None:
         _check_dev_tensor(lse, "lse", torch.float32, (T, num_heads))
+    if status is not None:
+        _check_dev_tensor(status, "status", torch.int32, (1,))
     if stream is None:
         stream = torch.cuda.current_stream(q_nope.device).cuda_stream
     dims = _Dims(num_heads, kv_lora_rank, rope_dim, page_size, num_pages, sm_scale)
@@ -462,7 +481,7 @@ def mla_run_noalloc(qo_indptr, kv_indptr, kv_indices, last_page_len, q_nope, q_p
         ctypes.c_void_p(q_nope.data_ptr()), ctypes.c_void_p(q_pe.data_ptr() if q_pe is not None else 0),
         ctypes.c_void_p(cache.data_ptr()),
         ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(lse.data_ptr() if lse is not None else 0),
-        ctypes.c_void_p(stream or 0))
+        ctypes.c_void_p(stream or 0), ctypes.c_void_p(status.data_ptr() if status is not None else 0))
     if st != MLA_OK:
         raise MlaError(st, "mla_run_noalloc")
 

@@ -240,8 +240,21 @@ static __device__ __align__(256) unsigned char g_mla_noalloc_scratch[kScratchByt
 extern "C" mla_status mla_run_noalloc(const mla_dims* dims, int32_t batch, const int32_t* qo_indptr,
                                       const int32_t* kv_indptr, const int32_t* kv_indices,
                                       const int32_t* last_page_len, int32_t causal, const void* q_nope,
-                                      const void* q_pe, const void* cache, void* out, float* lse, void* stream) {
+                                      const void* q_pe, const void* cache, void* out, float* lse, void* stream,
+                                      int32_t* status_out) {
   if (!dims || (causal != 0 && causal != 1)) return MLA_ERR_INVALID_ARGUMENT;
+  if (status_out && (reinterpret_cast<uintptr_t>(status_out) & 3u)) return MLA_ERR_INVALID_ARGUMENT;
+  // The copies below read the static host buffers at enqueue time; a graph captured
+  // here would keep pointing at them (and at the caller's page table) while its launch
+  // shapes stayed those of this step, so a replay could run another step's work list.
+  {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(static_cast<cudaStream_t>(stream), &cs) != cudaSuccess) {
+      cudaGetLastError();
+      return MLA_ERR_CUDA;
+    }
+    if (cs != cudaStreamCaptureStatusNone) return MLA_ERR_UNSUPPORTED;
+  }
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
@@ -269,7 +282,14 @@ extern "C" mla_status mla_run_noalloc(const mla_dims* dims, int32_t batch, const
   mla_status st = plan_fixed(*dims, batch, qo_indptr, kv_indptr, kv_indices, last_page_len, causal != 0,
                              g_dev[dev].num_sms, &n_work, &n_merge, &n_refs, &n_ws_rows, &T);
   if (st != MLA_OK) return st;
-  if (n_work == 0) return MLA_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (n_work == 0) {
+    if (status_out && cudaMemsetAsync(status_out, 0, sizeof(int32_t), s) != cudaSuccess) {
+      cudaGetLastError();
+      return MLA_ERR_CUDA;
+    }
+    return MLA_OK;
+  }
   const bool rope = dims->rope_dim > 0;  // without kpe, q_pe is not read (may be NULL)
   if (!q_nope || (rope && !q_pe) || !cache || !out) return MLA_ERR_INVALID_ARGUMENT;
   auto misaligned = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) != 0; };
@@ -280,7 +300,6 @@ extern "C" mla_status mla_run_noalloc(const mla_dims* dims, int32_t batch, const
   // Fill the scratch: status word cleared, work and merge lists, page-table copy.  The
   // copies read host memory that is pageable, so each returns once its source has been
   // read and the static host buffers may be reused by the next call.
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t n_idx = static_cast<size_t>(kv_indptr[batch]);
   if (cudaMemsetAsync(scratch + kOffStatus, 0, 256, s) != cudaSuccess ||
       cudaMemcpyAsync(scratch + kOffWork, g_work, sizeof(WorkItem) * n_work, cudaMemcpyHostToDevice, s) !=
@@ -323,6 +342,13 @@ extern "C" mla_status mla_run_noalloc(const mla_dims* dims, int32_t batch, const
     MergeParams mp{reinterpret_cast<const MergeItem*>(scratch + kOffMerge),
                    reinterpret_cast<const int32_t*>(scratch + kOffRefs), ap.ws_o, ap.ws_lse, out, lse};
     if (launch_merge(mp, n_merge, s) != cudaSuccess) return MLA_ERR_CUDA;
+  }
+  // The status word the kernels wrote (0, or MLA_ERR_DEVICE_TIMEOUT in its low byte),
+  // handed to the caller's own word once the stream has passed the launches.
+  if (status_out && cudaMemcpyAsync(status_out, scratch + kOffStatus, sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                                    s) != cudaSuccess) {
+    cudaGetLastError();
+    return MLA_ERR_CUDA;
   }
   return MLA_OK;
 }

@@ -56,23 +56,11 @@ struct QTile {
   int32_t first_out, n_out;  // output tiles covered (cascade tiles)
 };
 
-// Longest-processing-time-first makespan of `costs` over `units` identical units.  Stops
-// early (returning a value >= `give_up`) once the makespan cannot end below `give_up`.
-double lpt_makespan(std::vector<double>& costs, int units, double give_up) {
-  std::sort(costs.begin(), costs.end(), std::greater<double>());
-  std::priority_queue<double, std::vector<double>, std::greater<double>> load;
-  for (int i = 0; i < units; ++i) load.push(0.0);
-  double worst = 0.0;
-  for (double c : costs) {
-    double l = load.top();
-    load.pop();
-    l += c;
-    worst = std::max(worst, l);
-    if (worst >= give_up) return worst;
-    load.push(l);
-  }
-  return worst;
-}
+// Item costs are whole numbers of key-tile steps: a piece's key tiles plus the fixed
+// cost of an item, plus the extra of a partial result.
+constexpr int32_t kItemCostI = static_cast<int32_t>(kItemCost);
+constexpr int32_t kSplitCostI = static_cast<int32_t>(kSplitCost);
+static_assert(double(kItemCostI) == kItemCost && double(kSplitCostI) == kSplitCost, "integer item costs");
 
 // Pieces of at most `chunk` key tiles (sizes differing by at most one).
 inline int32_t pieces_for(int32_t ntiles, int32_t chunk) {
@@ -80,6 +68,112 @@ inline int32_t pieces_for(int32_t ntiles, int32_t chunk) {
   if (chunk <= 0) return 1;
   return (ntiles + chunk - 1) / chunk;
 }
+
+// ceil(ntiles / chunk) for 1 <= chunk, 0 <= ntiles < 2^24, from a float reciprocal
+// (one multiply, corrected to the exact quotient) instead of an integer division.
+struct PieceCounter {
+  int32_t chunk;
+  float inv;
+  explicit PieceCounter(int32_t c) : chunk(c), inv(1.0f / float(c)) {}
+  int32_t operator()(int32_t ntiles) const {
+    if (ntiles <= 0) return 1;
+    int32_t n = static_cast<int32_t>(float(ntiles) * inv);  // within one of ntiles / chunk
+    while (n * chunk < ntiles) ++n;
+    while (n > 1 && (n - 1) * chunk >= ntiles) --n;
+    return n;
+  }
+};
+
+// What a split size makes of the tiles, in one pass.
+struct SplitStats {
+  int64_t items = 0, partials = 0, ws_rows = 0;
+  int64_t total_cost = 0;  // sum of item costs
+  int32_t longest = 0;     // largest item cost
+};
+
+SplitStats stats_for(const std::vector<QTile>& tiles, int32_t chunk) {
+  SplitStats st;
+  if (chunk <= 0) {  // no split: one item per tile
+    for (const QTile& t : tiles) {
+      const int32_t fixed = kItemCostI + (t.must_merge ? kSplitCostI : 0);
+      st.items += 1;
+      st.total_cost += int64_t(t.ntiles) + fixed;
+      st.longest = std::max(st.longest, t.ntiles + fixed);
+      if (t.must_merge) {
+        st.partials += 1;
+        st.ws_rows += t.n_rows;
+      }
+    }
+    return st;
+  }
+  for (const QTile& t : tiles) {
+    const int32_t n = pieces_for(t.ntiles, chunk);
+    const bool part = n > 1 || t.must_merge;
+    const int32_t fixed = kItemCostI + (part ? kSplitCostI : 0);
+    st.items += n;
+    st.total_cost += int64_t(t.ntiles) + int64_t(n) * fixed;
+    st.longest = std::max(st.longest, (t.ntiles + n - 1) / n + fixed);
+    if (part) {
+      st.partials += n;
+      st.ws_rows += int64_t(n) * t.n_rows;
+    }
+  }
+  return st;
+}
+
+// The tiles counted by their number of key tiles, so that what a split size makes of
+// them is evaluated in time proportional to (longest tile / chunk) rather than to the
+// number of tiles.  Valid when no tile must merge (no cascade prefixes): then a tile's
+// pieces are partials exactly when it is cut.
+struct TileCounts {
+  int32_t max_nt = 0;
+  int64_t n = 0, sum_nt = 0;
+  std::vector<int64_t> gt;     // gt[x]: tiles with more than x key tiles, x in [0, max_nt]
+  std::vector<int32_t> le_max; // le_max[x]: the largest tile length <= x (-1 if none)
+
+  void build(const std::vector<QTile>& tiles, int32_t max_ntiles) {
+    max_nt = max_ntiles;
+    n = static_cast<int64_t>(tiles.size());
+    sum_nt = 0;
+    gt.assign(static_cast<size_t>(max_nt) + 2, 0);
+    le_max.assign(static_cast<size_t>(max_nt) + 1, -1);
+    for (const QTile& t : tiles) {
+      sum_nt += t.ntiles;
+      ++gt[t.ntiles];  // first the count of each length
+      le_max[t.ntiles] = t.ntiles;
+    }
+    int64_t above = 0;
+    for (int32_t x = max_nt; x >= 0; --x) {  // then suffix sums: tiles longer than x
+      const int64_t eq = gt[x];
+      gt[x] = above;
+      above += eq;
+    }
+    for (int32_t x = 1; x <= max_nt; ++x) le_max[x] = std::max(le_max[x], le_max[x - 1]);
+  }
+  // sum over j >= 1 of the tiles longer than j * c
+  int64_t cut_sum(int32_t c) const {
+    int64_t s = 0;
+    for (int64_t x = c; x <= max_nt; x += c) s += gt[x];
+    return s;
+  }
+  int64_t items(int32_t c) const { return n + cut_sum(c); }
+  SplitStats stats(int32_t c) const {
+    SplitStats st;
+    const int64_t cuts = cut_sum(c);
+    st.items = n + cuts;
+    st.partials = gt[c] + cuts;  // the pieces of the tiles longer than c
+    st.total_cost = sum_nt + kItemCostI * st.items + kSplitCostI * st.partials;
+    // a lower bound on the longest item: the longest uncut tile, and a piece of the
+    // longest tile if that one is cut
+    int32_t longest = le_max[std::min(c, max_nt)] >= 0 ? le_max[std::min(c, max_nt)] + kItemCostI : 0;
+    if (max_nt > c) {
+      const int32_t pieces = (max_nt + c - 1) / c;
+      longest = std::max(longest, (max_nt + pieces - 1) / pieces + kItemCostI + kSplitCostI);
+    }
+    st.longest = longest;
+    return st;
+  }
+};
 
 struct Counts {
   int64_t work = 0, merge = 0, refs = 0, ws_rows = 0, partials = 0;
@@ -109,7 +203,12 @@ Counts count_for(const std::vector<QTile>& tiles, int32_t n_out, int32_t chunk) 
   return c;
 }
 
-bool fits(const Counts& c, const PlanRequest& r) {
+bool bounded(const PlanRequest& r) { return r.max_work > 0 || r.max_merge > 0 || r.max_refs > 0 || r.max_ws_rows > 0; }
+
+// Whether a split size stays within a graph plan's bounds and the int32 workspace rows.
+bool fits(const std::vector<QTile>& tiles, int32_t n_out, int32_t chunk, const PlanRequest& r) {
+  if (!bounded(r)) return stats_for(tiles, chunk).ws_rows <= std::numeric_limits<int32_t>::max() - kTileM;
+  const Counts c = count_for(tiles, n_out, chunk);
   if (r.max_work > 0 && c.work > r.max_work) return false;
   if (r.max_merge > 0 && c.merge > r.max_merge) return false;
   if (r.max_refs > 0 && c.refs > r.max_refs) return false;
@@ -118,26 +217,55 @@ bool fits(const Counts& c, const PlanRequest& r) {
   return true;
 }
 
-double estimate(const std::vector<QTile>& tiles, int32_t chunk, int units,
+// Longest-processing-time-first makespan of the items a split size gives, over `units`
+// identical SM pairs, plus the merge pass (which reads every partial once, spread over
+// all units).  The costs are whole numbers no larger than `max_cost`, so they are sorted
+// by counting; the unit loads live in a binary min-heap.  Stops early (returning a value
+// >= `give_up`) once the makespan cannot end below `give_up`.
+double estimate(const std::vector<QTile>& tiles, int32_t chunk, int units, int32_t max_cost,
                 double give_up = std::numeric_limits<double>::infinity()) {
-  std::vector<double> costs;
-  costs.reserve(tiles.size() * 2);
+  static thread_local std::vector<int32_t> count;  // items per cost
+  static thread_local std::vector<int64_t> load;   // unit loads (min-heap)
+  count.assign(static_cast<size_t>(max_cost) + 1, 0);
   int64_t partials = 0;
   for (const QTile& t : tiles) {
     const int32_t n = pieces_for(t.ntiles, chunk);
-    if (n == 1 && !t.must_merge) {
-      costs.push_back(t.ntiles + kItemCost);
-    } else {
-      partials += n;
-      for (int32_t p = 0; p < n; ++p) {
-        const int32_t lo = (int64_t)t.ntiles * p / n, hi = (int64_t)t.ntiles * (p + 1) / n;
-        costs.push_back((hi - lo) + kItemCost + kSplitCost);
+    const bool part = n > 1 || t.must_merge;
+    const int32_t fixed = kItemCostI + (part ? kSplitCostI : 0);
+    // n pieces: ntiles % n of them one tile longer than the rest
+    const int32_t q = t.ntiles / n, r = t.ntiles % n;
+    if (r > 0) count[q + 1 + fixed] += r;
+    count[q + fixed] += n - r;
+    if (part) partials += n;
+  }
+  const double merge = kSplitCost * double(partials) / units;
+  const double limit = give_up - merge;
+  // The least loaded unit takes the next longest item: its load grows in place at the
+  // root of the heap, which is then sifted down.
+  load.assign(static_cast<size_t>(units), 0);  // all zero: already a heap
+  int64_t* h = load.data();
+  const int m = units;
+  int64_t worst = 0;
+  for (int32_t cost = max_cost; cost >= 0; --cost) {
+    for (int32_t k = count[cost]; k > 0; --k) {
+      const int64_t l = h[0] + cost;
+      if (l > worst) {
+        worst = l;
+        if (double(worst) >= limit) return double(worst) + merge;
       }
+      int i = 0;
+      for (;;) {
+        const int a = 2 * i + 1, b = a + 1;
+        if (a >= m) break;
+        const int c = (b < m && h[b] < h[a]) ? b : a;
+        if (h[c] >= l) break;
+        h[i] = h[c];
+        i = c;
+      }
+      h[i] = l;
     }
   }
-  // The merge pass reads every partial once, spread over all units.
-  const double merge = kSplitCost * double(partials) / units;
-  return lpt_makespan(costs, units, give_up - merge) + merge;
+  return double(worst) + merge;
 }
 
 }  // namespace
@@ -157,6 +285,8 @@ mla_status build_layout(const PlanRequest& req, PlanLayout* out) {
   if (!qo_indptr || !kv_indptr || (batch > 0 && !last_page_len)) return MLA_ERR_INVALID_ARGUMENT;
   if (req.split_keys > 0 && req.split_keys % kTileN != 0) return MLA_ERR_INVALID_ARGUMENT;
   const int32_t H = d.num_heads, P = d.page_size;
+  int log2_P = 0;  // page sizes are powers of two (shape_supported)
+  while ((1 << log2_P) < P) ++log2_P;
   if ((int64_t)d.num_pages * P > std::numeric_limits<int32_t>::max())
     return MLA_ERR_INVALID_ARGUMENT;
 
@@ -174,7 +304,14 @@ mla_status build_layout(const PlanRequest& req, PlanLayout* out) {
     if (kv_indices[i] < 0 || kv_indices[i] >= d.num_pages) return MLA_ERR_INVALID_ARGUMENT;
 
   // --- per-row key counts (k_b from the tables; c_b = k_b - q_b attended if context-only)
-  std::vector<int32_t> k_full(batch, 0);
+  // Working arrays live in per-thread scratch that keeps its capacity from call to call,
+  // so planning a step of a size seen before allocates nothing but the plan's own lists.
+  static thread_local std::vector<int32_t> k_full, row_first_tile, suffix_from, ref_count, ref_next;
+  static thread_local std::vector<uint8_t> out_cascaded;
+  static thread_local std::vector<QTile> outs, tiles;
+  static thread_local std::vector<uint64_t> order;
+  static thread_local std::vector<WorkItem> sorted;
+  k_full.assign(batch, 0);
   out->kv_len.assign(batch, 0);
   for (int32_t b = 0; b < batch; ++b) {
     const int64_t n = kv_indptr[b + 1] - kv_indptr[b];
@@ -208,15 +345,38 @@ mla_status build_layout(const PlanRequest& req, PlanLayout* out) {
         out->append_ok = false;
         continue;
       }
-      const int32_t page = kv_indices[kv_indptr[b] + pos / P];
-      out->append_rows[qo_indptr[b] + i] = page * P + static_cast<int32_t>(pos % P);
+      const int32_t page = kv_indices[kv_indptr[b] + (pos >> log2_P)];
+      out->append_rows[qo_indptr[b] + i] = page * P + static_cast<int32_t>(pos & (P - 1));
+    }
+  }
+  // A page listed twice can give two tokens one slot.  The later token's row is the one
+  // kept: earlier tokens naming a slot that a later token also names get no destination,
+  // so no two threads of the append ever store to one slot (their 16-byte pieces could
+  // otherwise interleave).  Tokens are visited last to first against a hash set of the
+  // slots already claimed.
+  if (T > 1) {
+    static thread_local std::vector<int32_t> seen;
+    size_t cap = 16;
+    while (cap < 2 * static_cast<size_t>(T)) cap <<= 1;
+    if (seen.size() < cap) seen.resize(cap);
+    std::fill(seen.begin(), seen.begin() + cap, -1);
+    const size_t mask = cap - 1;
+    for (int64_t t = T - 1; t >= 0; --t) {
+      const int32_t row = out->append_rows[t];
+      if (row < 0) continue;
+      size_t h = (static_cast<uint32_t>(row) * 2654435761u) & mask;
+      while (seen[h] >= 0 && seen[h] != row) h = (h + 1) & mask;
+      if (seen[h] == row)
+        out->append_rows[t] = -1;  // a later token writes this slot
+      else
+        seen[h] = row;
     }
   }
 
   // --- output tiles: 128 / H consecutive tokens of one row, all heads
   const int32_t tok_per_tile = kTileM / H;
-  std::vector<QTile> outs;  // one per output tile, keys from 0
-  std::vector<int32_t> row_first_tile(batch + 1, 0);
+  outs.clear();  // one per output tile, keys from 0
+  row_first_tile.assign(batch + 1, 0);
   for (int32_t b = 0; b < batch; ++b) {
     row_first_tile[b] = static_cast<int32_t>(outs.size());
     const int32_t q_b = qo_indptr[b + 1] - qo_indptr[b];
@@ -242,9 +402,9 @@ mla_status build_layout(const PlanRequest& req, PlanLayout* out) {
   const int32_t n_out = static_cast<int32_t>(outs.size());
 
   // --- cascade: groups of consecutive rows sharing leading page ids
-  std::vector<QTile> tiles;  // what gets split: cascade tiles and per-row (suffix) tiles
-  std::vector<int32_t> suffix_from(n_out, 0);  // first key of each output tile's own item
-  std::vector<bool> out_cascaded(n_out, false);
+  tiles.clear();  // what gets split: cascade tiles and per-row (suffix) tiles
+  suffix_from.assign(n_out, 0);  // first key of each output tile's own item
+  out_cascaded.assign(n_out, 0);
   int32_t num_cascade_tiles = 0;
   if (req.cascade) {
     int32_t g = 0;
@@ -294,7 +454,7 @@ mla_status build_layout(const PlanRequest& req, PlanLayout* out) {
             // same queries as that tile would, and only adds a merge: leave it out.
             if (c.n_out < 2) continue;
             for (int32_t oo = c.first_out; oo < c.first_out + c.n_out; ++oo) {
-              out_cascaded[oo] = true;
+              out_cascaded[oo] = 1;
               suffix_from[oo] = static_cast<int32_t>(s);
             }
             c.page_base = kv_indptr[g];
@@ -332,68 +492,96 @@ mla_status build_layout(const PlanRequest& req, PlanLayout* out) {
 
   // --- choose the split size (within a graph plan's bounds)
   const int units = std::max(1, req.num_sms / 2);
+  const int32_t max_cost = max_ntiles + kItemCostI + kSplitCostI;
   int32_t chunk = 0;  // 0: no split
   if (req.split_keys > 0) {
     chunk = req.split_keys / kTileN;
-    if (!fits(count_for(tiles, n_out, chunk), req)) return MLA_ERR_INVALID_ARGUMENT;
+    if (!fits(tiles, n_out, chunk, req)) return MLA_ERR_INVALID_ARGUMENT;
   } else {
-    if (!fits(count_for(tiles, n_out, 0), req)) return MLA_ERR_INVALID_ARGUMENT;
+    if (!fits(tiles, n_out, 0, req)) return MLA_ERR_INVALID_ARGUMENT;
     const double avg = (double(total_key_tiles) + kItemCost * tiles.size()) / units;
     // No split can help when the longest tile already fits in the average load of a pair.
     if (req.split_keys == 0 && !tiles.empty() && max_ntiles > 1 && max_ntiles + kItemCost > avg) {
-      // Every chunk size is a candidate (at most ~1000 of them, evenly spaced).
-      std::vector<int32_t> cands;
-      const int32_t stride = std::max<int32_t>(1, (max_ntiles - 2) / 1024);
-      for (int32_t c = 2; c < max_ntiles; c += stride) cands.push_back(c);
-      // Finalists for the full LPT estimate: for each number of waves k (items in k x
-      // pairs), the smallest chunk whose items still fit in k waves (the finest split
-      // with no straggling last wave), and the two candidates with the lowest bound on
-      // the makespan (the largest of: the longest item, the average load per pair, and
-      // the items some pair must take times the shortest item; plus the merge pass).
-      struct Scored {
+      // Items are dispatched to the SM pairs longest first, and a split pays when its
+      // items fill whole waves of pairs.  The candidates are therefore, for each number
+      // of waves k, the finest split whose items still fit in k waves (the number of
+      // items does not grow with the chunk size, so a bisection finds it).  Each is
+      // scored by the list-scheduling model, in order of a lower bound on its makespan
+      // (the longest item and the average load per pair, plus the merge pass), and a
+      // split is kept only if it is 1% better than the best so far.
+      struct Cand {
         double bound;
         int32_t chunk;
-        int64_t items;
       };
-      std::vector<Scored> scored;
-      for (int32_t c : cands) {
-        double longest = 0.0, shortest = std::numeric_limits<double>::infinity(), sum = 0.0, partials = 0.0;
-        int64_t items = 0;
-        for (const QTile& t : tiles) {
-          const int32_t n = pieces_for(t.ntiles, c);
-          const bool part = n > 1 || t.must_merge;
-          const double fixed = kItemCost + (part ? kSplitCost : 0.0);
-          longest = std::max(longest, double((t.ntiles + n - 1) / n) + fixed);
-          shortest = std::min(shortest, double(t.ntiles / n) + fixed);
-          sum += t.ntiles + n * fixed;
-          items += n;
-          if (part) partials += n;
-        }
-        const double per_unit = double((items + units - 1) / units) * shortest;
-        scored.push_back(Scored{std::max({longest, sum / units, per_unit}) + kSplitCost * partials / units, c, items});
-      }
-      std::vector<int32_t> finalists;
+      Cand cands[kMaxWaves + 3];
+      int n_cands = 0;
+      bool any_must = false;
+      for (const QTile& t : tiles) any_must |= t.must_merge;
+      static thread_local TileCounts hist;
+      if (!any_must) hist.build(tiles, max_ntiles);
+      auto stats = [&](int32_t c) { return any_must ? stats_for(tiles, c) : hist.stats(c); };
+      auto add = [&](int32_t c) {
+        if (c < 2 || c >= max_ntiles) return;
+        for (int i = 0; i < n_cands; ++i)
+          if (cands[i].chunk == c) return;
+        const SplitStats st = stats(c);
+        const double bound = std::max(double(st.longest), double(st.total_cost) / units) +
+                             kSplitCost * double(st.partials) / units;
+        cands[n_cands++] = Cand{bound, c};
+      };
+      int32_t prev = -1;
       for (int64_t k = 1; k <= kMaxWaves; ++k) {
-        // cands ascend, items descend: the first candidate within k waves
-        for (const Scored& x : scored)
-          if (x.items <= k * units) {
-            if (finalists.empty() || finalists.back() != x.chunk) finalists.push_back(x.chunk);
-            break;
+        int32_t lo = 2, hi = (prev > 0 ? prev : max_ntiles) - 1, found = -1;
+        while (lo <= hi) {
+          const int32_t mid = lo + (hi - lo) / 2;
+          int64_t items = 0;
+          if (any_must) {
+            const PieceCounter pieces(mid);
+            for (const QTile& t : tiles) items += pieces(t.ntiles);
+          } else {
+            items = hist.items(mid);
           }
+          if (items <= k * units) {
+            found = mid;
+            hi = mid - 1;
+          } else {
+            lo = mid + 1;
+          }
+        }
+        if (found < 0 || found == prev) continue;
+        prev = found;
+        add(found);
       }
-      std::sort(scored.begin(), scored.end(), [](const Scored& x, const Scored& y) { return x.bound < y.bound; });
-      for (size_t i = 0; i < scored.size() && i < 2; ++i) finalists.push_back(scored[i].chunk);
-      std::sort(finalists.begin(), finalists.end(), std::greater<int32_t>());
-      finalists.erase(std::unique(finalists.begin(), finalists.end()), finalists.end());
-      double best = estimate(tiles, 0, units);
-      for (int32_t c : finalists) {
-        if (!fits(count_for(tiles, n_out, c), req)) continue;
-        // (an estimate that cannot beat best * 0.99 stops early: prefer fewer splits
-        // unless clearly better)
-        const double e = estimate(tiles, c, units, best * 0.99);
+      // ... and the balance point, where the longest item stops being shorter than the
+      // average load of a pair (the chunk that minimises the lower bound), with its
+      // neighbours: between whole waves the model can still prefer a split there.
+      {
+        int32_t lo = 2, hi = max_ntiles - 1, found = -1;
+        while (lo <= hi) {
+          const int32_t mid = lo + (hi - lo) / 2;
+          const SplitStats st = stats(mid);
+          if (double(st.longest) >= double(st.total_cost) / units) {
+            found = mid;
+            hi = mid - 1;
+          } else {
+            lo = mid + 1;
+          }
+        }
+        if (found > 0) {
+          add(found - 1);
+          add(found);
+          add(found + 1);
+        }
+      }
+      std::sort(cands, cands + n_cands, [](const Cand& x, const Cand& y) { return x.bound < y.bound; });
+      double best = estimate(tiles, 0, units, max_cost);
+      for (int i = 0; i < n_cands; ++i) {
+        if (cands[i].bound >= best * 0.99) break;  // neither this nor any later one can win
+        if (!fits(tiles, n_out, cands[i].chunk, req)) continue;
+        const double e = estimate(tiles, cands[i].chunk, units, max_cost, best * 0.99);
         if (e < best * 0.99) {
           best = e;
-          chunk = c;
+          chunk = cands[i].chunk;
         }
       }
     }
@@ -422,7 +610,7 @@ mla_status build_layout(const PlanRequest& req, PlanLayout* out) {
         int64_t it = 0;
         const double l = latency(c, &it);
         if (it > units) break;  // finer splits only add items
-        if (l < best_lat * 0.99 && fits(count_for(tiles, n_out, c), req)) {
+        if (l < best_lat * 0.99 && fits(tiles, n_out, c, req)) {
           best_lat = l;
           chunk = c;
         }
@@ -431,17 +619,49 @@ mla_status build_layout(const PlanRequest& req, PlanLayout* out) {
   }
   out->chunk_tiles = chunk;
 
-  // --- emit items and the merge references of every output tile
-  out->work.clear();
+  // --- emit items and the merge references of every output tile.  Each output tile's
+  // references are its partials in emission order; they are counted first, so that the
+  // merge list and the reference list are written in place.
+  ref_count.assign(n_out, 0);
+  int64_t n_items = 0;
+  for (const QTile& t : tiles) {
+    const int32_t n = pieces_for(t.ntiles, chunk);
+    n_items += n;
+    if (n == 1 && !t.must_merge) continue;
+    if (t.cascade) {
+      for (int32_t o = t.first_out; o < t.first_out + t.n_out; ++o) ref_count[o] += n;
+    } else {
+      ref_count[t.out_tile] += n;
+    }
+  }
   out->merge.clear();
-  out->refs.clear();
-  std::vector<std::vector<int32_t>> refs_of(n_out);
+  ref_next.resize(n_out);
+  int32_t n_refs = 0;
+  for (int32_t o = 0; o < n_out; ++o) {
+    ref_next[o] = n_refs;
+    if (ref_count[o] == 0) continue;
+    out->merge.push_back(MergeItem{outs[o].q_row0, outs[o].n_rows, n_refs, ref_count[o]});
+    n_refs += ref_count[o];
+  }
+  out->refs.resize(n_refs);
+  sorted.resize(static_cast<size_t>(n_items));
   int32_t ws_row = 0, partials = 0, cascade_items = 0;
+  size_t wi = 0;
   for (const QTile& t : tiles) {
     const int32_t n = pieces_for(t.ntiles, chunk);
     const bool part = n > 1 || t.must_merge;
+    // piece p covers key tiles [floor(ntiles * p / n), floor(ntiles * (p + 1) / n)),
+    // stepped exactly without a division per piece: ntiles = q * n + r
+    const int32_t q = t.ntiles / n, r = t.ntiles % n;
+    int32_t hi = 0, rem = 0;
     for (int32_t p = 0; p < n; ++p) {
-      const int32_t lo = (int64_t)t.ntiles * p / n, hi = (int64_t)t.ntiles * (p + 1) / n;
+      const int32_t lo = hi;
+      hi = lo + q;
+      rem += r;
+      if (rem >= n) {
+        rem -= n;
+        ++hi;
+      }
       WorkItem w{t.q_row0, t.n_rows, t.page_base, t.kv_len, t.key0 + lo * kTileN,
                  std::min(t.key0 + hi * kTileN, t.vis_hi), t.diag_base, -1};
       if (t.ntiles == 0) w.key_begin = w.key_end = t.key0;
@@ -449,30 +669,47 @@ mla_status build_layout(const PlanRequest& req, PlanLayout* out) {
         w.partial = ws_row;
         if (t.cascade) {
           for (int32_t o = t.first_out; o < t.first_out + t.n_out; ++o)
-            refs_of[o].push_back(ws_row + (outs[o].q_row0 - t.q_row0));
+            out->refs[ref_next[o]++] = ws_row + (outs[o].q_row0 - t.q_row0);
         } else {
-          refs_of[t.out_tile].push_back(ws_row);
+          out->refs[ref_next[t.out_tile]++] = ws_row;
         }
         ws_row += t.n_rows;
         ++partials;
       }
       if (t.cascade) ++cascade_items;
-      out->work.push_back(w);
+      sorted[wi++] = w;
     }
-  }
-  for (int32_t o = 0; o < n_out; ++o) {
-    if (refs_of[o].empty()) continue;
-    out->merge.push_back(MergeItem{outs[o].q_row0, outs[o].n_rows, static_cast<int32_t>(out->refs.size()),
-                                   static_cast<int32_t>(refs_of[o].size())});
-    out->refs.insert(out->refs.end(), refs_of[o].begin(), refs_of[o].end());
   }
   out->num_partials = partials;
   out->ws_rows = ws_row;
   out->num_cascade = cascade_items;
-  // longest first; equal lengths keep their order, so a group's prefix items stay adjacent
-  std::stable_sort(out->work.begin(), out->work.end(), [](const WorkItem& a, const WorkItem& b) {
-    return (a.key_end - a.key_begin) > (b.key_end - b.key_begin);
-  });
+  // Longest first; equal lengths keep their order, so a group's prefix items stay
+  // adjacent.  Sorted as (length descending, emission index) keys: a total order, so the
+  // result is the stable order without a stable sort's buffer.
+  order.resize(sorted.size());
+  for (size_t i = 0; i < sorted.size(); ++i) {
+    const uint32_t len = static_cast<uint32_t>(sorted[i].key_end - sorted[i].key_begin);
+    order[i] = (uint64_t(~len) << 32) | uint64_t(i);
+  }
+  if (order.size() <= 512) {
+    std::sort(order.begin(), order.end());
+  } else {
+    // Many items (prefill steps): a least-significant-digit radix sort on the 32-bit
+    // length key, 11 bits a pass; each pass is stable, and the keys are built in
+    // emission order, so equal lengths keep that order.
+    static thread_local std::vector<uint64_t> tmp;
+    tmp.resize(order.size());
+    for (int shift = 32; shift < 64; shift += 11) {
+      size_t count[2049] = {0};
+      for (uint64_t k : order) ++count[((k >> shift) & 2047) + 1];
+      if (count[((order[0] >> shift) & 2047) + 1] == order.size()) continue;  // one digit: no-op
+      for (int i = 0; i < 2048; ++i) count[i + 1] += count[i];
+      for (uint64_t k : order) tmp[count[(k >> shift) & 2047]++] = k;
+      order.swap(tmp);
+    }
+  }
+  out->work.resize(sorted.size());
+  for (size_t i = 0; i < order.size(); ++i) out->work[i] = sorted[static_cast<uint32_t>(order[i])];
   return MLA_OK;
 }
 

@@ -12,6 +12,7 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 import paged_head_latent_mla_b200 as M  # noqa: E402
+from workloads import make_config  # noqa: E402
 
 SCALE = 192 ** -0.5
 
@@ -165,3 +166,69 @@ def test_plain_c_client(tmp_path):
     assert got["run_host_only"] == str(M.MLA_ERR_INVALID_ARGUMENT)
     assert got["merge_state_bad"] == str(M.MLA_ERR_INVALID_ARGUMENT)
     assert "done" in got
+
+
+def test_cache_shape_checked_before_any_launch():
+    """The binding refuses a cache tensor with fewer pages than the plan declares, another
+    page size or another row width before it reaches the library (the kernels' tensor
+    maps span num_pages * page_size rows, so a smaller tensor would be read past its
+    end).  Checked with CPU tensors: the shape check comes before the device checks."""
+    import torch
+
+    d = make_config("tiny_decode", tables_only=True)
+    p = M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=d.num_heads,
+                   page_size=d.page_size, num_pages=d.num_pages, sm_scale=d.sm_scale, host_only=True)
+    T, H = int(d.qo_indptr[-1]), d.num_heads
+    qn = torch.zeros((T, H, 512), dtype=torch.bfloat16)
+    qp = torch.zeros((T, H, 64), dtype=torch.bfloat16)
+    for shape in [(d.num_pages - 1, d.page_size, 576), (d.num_pages, d.page_size * 2, 576),
+                  (d.num_pages, d.page_size, 512), (d.num_pages * d.page_size, 576)]:
+        cache = torch.zeros(shape, dtype=torch.bfloat16)
+        with pytest.raises(ValueError, match="cache must have shape"):
+            M.mla_run(p, qn, qp, cache)
+        with pytest.raises(ValueError, match="cache must have shape"):
+            M.mla_append_kv(p, torch.zeros((T, 576), dtype=torch.bfloat16), cache)
+        with pytest.raises(ValueError, match="cache must have shape"):
+            M.mla_run_noalloc(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, qn, qp, cache,
+                              torch.zeros((T, H, 512), dtype=torch.bfloat16), num_heads=H,
+                              page_size=d.page_size, num_pages=d.num_pages, sm_scale=d.sm_scale)
+    p.destroy()
+
+
+def _write_tables(path, steps):
+    """One or two steps' tables in the int32 layout tests/c/plan_timer.cpp reads."""
+    with open(path, "wb") as f:
+        for d in steps:
+            hdr = np.array([d.num_heads, d.page_size, d.num_pages, d.batch, 1 if d.causal else 0], np.int32)
+            for a in (hdr, d.qo_indptr.numpy(), d.kv_indptr.numpy(), d.kv_indices.numpy(), d.last_page_len.numpy()):
+                f.write(np.ascontiguousarray(a, dtype=np.int32).tobytes())
+
+
+def test_plan_timer_cpp_client(tmp_path):
+    """The C++ planning timer (the same client the benchmark runs on the GPU machine) builds
+    against include/mla.h, links the library and times host-only plans of the batch-64
+    decode step: fresh plans, unchanged updates (recognised, nothing re-planned) and
+    changed updates.  The numbers are reported, not asserted: this host is not the
+    benchmark's."""
+    import shutil
+    import subprocess
+
+    cxx = shutil.which("g++") or shutil.which("c++")
+    if cxx is None:
+        pytest.skip("no C++ compiler")
+    lib_dir = os.path.dirname(M.LIB_PATH)
+    exe = str(tmp_path / "plan_timer")
+    r = subprocess.run([cxx, "-O2", "-std=c++17", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        os.path.join(ROOT, "tests", "c", "plan_timer.cpp"), "-L", lib_dir, "-l:libmla_b200.so",
+                        "-Wl,-rpath," + lib_dir, "-o", exe], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    tables = str(tmp_path / "decode_b64.tables")
+    _write_tables(tables, [make_config("decode_b64", tables_only=True),
+                           make_config("decode_b64", seed=1, tables_only=True)])
+    r = subprocess.run([exe, tables, "50", "1"], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    got = {k: float(v) for k, v in (line.split() for line in r.stdout.strip().splitlines())}
+    assert set(got) == {"fresh", "update_same", "update_changed"}
+    assert all(v > 0 for v in got.values())
+    assert got["update_same"] < got["update_changed"]  # an unchanged step is only compared
+    print("host-only planning, decode_b64 (us):", got)

@@ -87,6 +87,58 @@ def test_run_append_attends_the_appended_rows():
     plan.destroy()
 
 
+def _slot_writers(d, page_size):
+    """For every (page, slot) the step's tokens write, the tokens that name it (the
+    oracle's key-to-slot mapping: token i of row b is key k_b - q_b + i)."""
+    qo = d.qo_indptr.numpy()
+    k_all = O.kv_lengths(d.kv_indptr, d.last_page_len, page_size)
+    writers = {}
+    for b in range(len(qo) - 1):
+        q_b = int(qo[b + 1] - qo[b])
+        for i in range(q_b):
+            loc = O.key_location(d.kv_indptr, d.kv_indices, page_size, b, int(k_all[b]) - q_b + i)
+            writers.setdefault(loc, []).append(int(qo[b]) + i)
+    return writers
+
+
+def test_append_two_tokens_on_one_slot_leaves_one_of_them():
+    """Two tokens whose positions name the same cache slot (a page listed twice: across
+    two rows that share their last page, and within one row whose list repeats a page).
+    The method leaves one of the tokens' rows there without fixing which; the check
+    accepts exactly those, then checks the library's stated choice (the latest token).
+    Every slot named once holds its token's row exactly, and every other slot is
+    unchanged."""
+    P = 16
+    d = make_custom([1, 1, 17, 2], [70, 70, 17, 40], 64, P, seed=66, extra_pool_pages=3)
+    idx = d.kv_indices.clone()
+    kvp = d.kv_indptr.numpy()
+    idx[kvp[1]:kvp[2]] = idx[kvp[0]:kvp[1]]  # row 1 names row 0's pages: both last tokens hit one slot
+    idx[kvp[2] + 1] = idx[kvp[2]]            # row 2 (17 keys, 17 tokens) lists its page twice
+    d.kv_indices = idx
+    T = int(d.qo_indptr[-1])
+    kv_new = _kv_new(T, 67)
+    plan = _plan(d)
+    cache = d.cache.to(DEV)
+    M.mla_append_kv(plan, kv_new.to(DEV), cache)
+    torch.cuda.synchronize()
+    plan.destroy()
+    got = cache.cpu()
+    new = kv_new
+    writers = _slot_writers(d, P)
+    assert any(len(t) > 1 for t in writers.values())
+    touched = torch.zeros(got.shape[:2], dtype=torch.bool)
+    for (page, slot), toks in writers.items():
+        touched[page, slot] = True
+        row = got[page, slot]
+        assert any(torch.equal(row, new[t]) for t in toks), f"slot ({page}, {slot}) holds none of tokens {toks}"
+    assert torch.equal(got[~touched], d.cache[~touched])
+    # the library keeps the latest token's row (its plan drops the earlier writes), which
+    # is also what the oracle's scatter in token order leaves
+    ref = torch.from_numpy(O.append_latent(d.cache, kv_new, d.qo_indptr, d.kv_indptr, d.kv_indices,
+                                           d.last_page_len, P)).to(torch.bfloat16)
+    assert torch.equal(ref, got)
+
+
 def test_append_rejects_rows_without_slots():
     d = make_custom([5], [3], 128, 64, seed=65)
     plan = _plan(d)
