@@ -193,6 +193,17 @@ def oracle_sample(d, budget_s: float, max_rows=None):
     return dt, kvb, done, threads
 
 
+L2_NOTE = ("GPU arm: inputs rotated over HBM copies (at least 3x L2 in total where memory allows), never "
+           "L2-resident between steps")
+
+
+def config_of(name, d):
+    """The workload description both arms print (identical dicts for the same workload)."""
+    w = work_of(d)
+    return {"workload": name, "description": d.description, "kv_bytes_per_step": w["kv_bytes"],
+            "flops_per_step": w["flops"], "l2": L2_NOTE}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -216,7 +227,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "description": d.description},
+        "config": config_of(args.workload, d),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
                          "sample": f"each step: the first {rows} rows of {args.workload} (all their queries), "
                                    f"fp64 NumPy oracle, ~{per_step:.1f} s budget"},
@@ -231,7 +242,7 @@ def make_runner(d, device, n_copies, timing=True, plan_kw=None):
     """Plan once; keep `n_copies` copies of the inputs in HBM and rotate through them so
     consecutive steps never find their inputs in L2.  With `timing` the plan records CUDA
     events around each of its launches (kernel durations for the roofline); those events
-    sit between the attention and merge launches, so headline steps use a plan without."""
+    sit between the attention and merge launches."""
     import ctypes
 
     import torch
@@ -269,9 +280,16 @@ def input_bytes(d):
 
 
 def time_workload(d, device, steps, warmup, dist=None, soak_s=0.0, sampler=None, copies=0, plan_kw=None):
-    """Two timed regions over the same resident inputs: K steps through a plain plan (the
-    product path: the step value), then K steps through a plan that records events
-    around each launch (the per-kernel durations for the roofline)."""
+    """Time K steps of the workload on resident inputs.
+
+    The timed region runs the steps through a plan that records CUDA events around each
+    of its launches (before the attention kernel, between it and the merge kernel, after
+    the merge), so the step time and the per-kernel durations come from the same K steps
+    under the same clocks: a kernel can never read longer than the step that contains it.
+    The region is bracketed by a barrier and a device synchronise and timed with CUDA
+    events on the launch stream.  Afterwards the same K steps run once more through a
+    plain plan (no events between the launches, the merge set up while the attention
+    drains): the product path's own step time, reported beside the headline."""
     import torch
 
     import paged_head_latent_mla_b200 as M
@@ -280,29 +298,29 @@ def time_workload(d, device, steps, warmup, dist=None, soak_s=0.0, sampler=None,
     free, _ = torch.cuda.mem_get_info(device)
     while n_copies > 1 and n_copies * input_bytes(d) > 0.6 * free:
         n_copies -= 1
-    plan, step, out, lse, copies = make_runner(d, device, n_copies, timing=False, plan_kw=plan_kw)
-    tplan = M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=d.num_heads,
-                       page_size=d.page_size, num_pages=d.num_pages, sm_scale=d.sm_scale, causal=d.causal,
-                       debug_flags=M.MLA_DEBUG_KERNEL_TIMING, **(plan_kw or {}))
+    tplan, tstep, out, lse, copies_ = make_runner(d, device, n_copies, timing=True, plan_kw=plan_kw)
+    plan = M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=d.num_heads,
+                      page_size=d.page_size, num_pages=d.num_pages, sm_scale=d.sm_scale, causal=d.causal,
+                      **(plan_kw or {}))
     lib = M.load_library()
     import ctypes
     stream = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
-    targs = [(tplan.handle, ctypes.c_void_p(qn.data_ptr()), ctypes.c_void_p(qp.data_ptr()),
+    pargs = [(plan.handle, ctypes.c_void_p(qn.data_ptr()), ctypes.c_void_p(qp.data_ptr()),
               ctypes.c_void_p(c.data_ptr()), ctypes.c_void_p(out.data_ptr()),
-              ctypes.c_void_p(lse.data_ptr() if lse is not None else 0), stream) for (qn, qp, c) in copies]
-    tstate = {"i": 0}
+              ctypes.c_void_p(lse.data_ptr() if lse is not None else 0), stream) for (qn, qp, c) in copies_]
+    pstate = {"i": 0}
 
-    def tstep():
-        a_ = targs[tstate["i"] % len(targs)]
-        tstate["i"] += 1
+    def pstep():
+        a_ = pargs[pstate["i"] % len(pargs)]
+        pstate["i"] += 1
         st_ = lib.mla_run(*a_)
         if st_ != 0:
             raise M.MlaError(st_, "mla_run")
 
-    info = M.mla_plan_get_info(plan)
+    info = M.mla_plan_get_info(tplan)
     for _ in range(warmup):
-        step()
         tstep()
+        pstep()
     torch.cuda.synchronize(device)
     for pl in (plan, tplan):
         st = M.mla_plan_check(pl)
@@ -310,11 +328,11 @@ def time_workload(d, device, steps, warmup, dist=None, soak_s=0.0, sampler=None,
             raise M.MlaError(st, "warm-up")
     if sampler is not None:
         sampler.start()
-    if soak_s > 0:  # untimed: lets the clock sampler see the GPU under this load
+    if soak_s > 0:  # untimed: brings the clocks to their level under this load, sampled
         t_end = time.perf_counter() + soak_s
         while time.perf_counter() < t_end:
             for _ in range(20):
-                step()
+                tstep()
             torch.cuda.synchronize(device)
     if dist is not None:
         dist.barrier()
@@ -323,29 +341,33 @@ def time_workload(d, device, steps, warmup, dist=None, soak_s=0.0, sampler=None,
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(steps):
-        step()
+        tstep()
     e1.record()
     torch.cuda.synchronize(device)
     if dist is not None:
         dist.barrier()
-    ms = e0.elapsed_time(e1)
-    # second region: per-kernel durations (events between the launches)
-    for _ in range(steps):
-        tstep()
-    torch.cuda.synchronize(device)
     clocks = sampler.stop() if sampler is not None else None
+    ms = e0.elapsed_time(e1)
     attn_ms, merge_ms = M.mla_plan_kernel_times(tplan, capacity=min(steps, 256))
+    # the product path without events between its launches, same steps, right after
+    e0.record()
+    for _ in range(steps):
+        pstep()
+    e1.record()
+    torch.cuda.synchronize(device)
+    ms_plain = e0.elapsed_time(e1)
     for pl in (plan, tplan):
         st = M.mla_plan_check(pl)
         if st != 0:
             raise M.MlaError(st, "timed steps")
-    res = {"ms_total": ms, "ms_per_step": ms / steps, "attn_ms": float(attn_ms.mean()),
+    res = {"ms_total": ms, "ms_per_step": ms / steps, "ms_per_step_plain": ms_plain / steps,
+           "attn_ms": float(attn_ms.mean()),
            "attn_ms_median": float(statistics.median(attn_ms.tolist())), "attn_ms_min": float(attn_ms.min()),
            "merge_ms": float(merge_ms.mean()), "info": info, "n_copies": n_copies, "clocks": clocks,
            "launches": steps * (1 + (1 if info["num_merge"] > 0 else 0))}
     plan.destroy()
     tplan.destroy()
-    del copies, out, lse
+    del copies_, out, lse
     torch.cuda.empty_cache()
     return res
 
@@ -451,6 +473,7 @@ def summarise(d, res, peaks):
     a = res["attn_ms"] * 1e-3
     return {
         "us_per_step": res["ms_per_step"] * 1e3,
+        "us_per_step_plain": res["ms_per_step_plain"] * 1e3,
         "attn_kernel_us": res["attn_ms"] * 1e3,
         "attn_kernel_us_median": res["attn_ms_median"] * 1e3,
         "attn_kernel_us_min": res["attn_ms_min"] * 1e3,
@@ -465,6 +488,7 @@ def summarise(d, res, peaks):
         "split_tiles": res["info"]["num_merge"],
         "kv_bytes": w["kv_bytes"],
         "flops": w["flops"],
+        "clocks": res.get("clocks"),
     }
 
 
@@ -660,8 +684,48 @@ def measure_next_rows(device, peaks):
     plan.destroy()
     res["plan_reuse_decode_b64"] = {"unchanged_update_us": reuse_us, "changed_update_us": replan_us,
                                     "fresh_plan_us": fresh_us,
-                                    "note": "host wall time per call, from numpy tables (binding included)"}
+                                    "cpp": plan_timer_cpp(d, d2),
+                                    "note": "host wall time per call, from numpy tables (binding included); "
+                                            "'cpp': the same calls from a C++ client of the C ABI"}
     return res
+
+
+def plan_timer_cpp(d, d2, iters=200):
+    """Host time of mla_plan / mla_plan_update on the steps' tables, measured by the C++
+    client tests/c/plan_timer.cpp through the C ABI (real plans on the current device:
+    uploads enqueued, no synchronisation).  None if no C++ compiler is at hand."""
+    import shutil
+
+    import numpy as np
+
+    cxx = shutil.which("g++") or shutil.which("c++")
+    if cxx is None:
+        return None
+    pkg = os.path.join(ROOT, "paged_head_latent_mla_b200")
+    with tempfile.TemporaryDirectory() as tmp:
+        exe = os.path.join(tmp, "plan_timer")
+        r = subprocess.run([cxx, "-O2", "-std=c++17", "-I", os.path.join(ROOT, "include"),
+                            os.path.join(ROOT, "tests", "c", "plan_timer.cpp"), "-L", pkg, "-l:libmla_b200.so",
+                            "-Wl,-rpath," + pkg, "-o", exe], capture_output=True, text=True)
+        if r.returncode != 0:
+            return {"error": r.stderr[-300:]}
+        tables = os.path.join(tmp, "steps.tables")
+        with open(tables, "wb") as f:
+            for x in (d, d2):
+                hdr = np.array([x.num_heads, x.page_size, max(d.num_pages, d2.num_pages), x.batch,
+                                1 if x.causal else 0], np.int32)
+                for a in (hdr, x.qo_indptr.numpy(), x.kv_indptr.numpy(), x.kv_indices.numpy(),
+                          x.last_page_len.numpy()):
+                    f.write(np.ascontiguousarray(a, dtype=np.int32).tobytes())
+        env = dict(os.environ)
+        r = subprocess.run([exe, tables, str(iters), "0"], capture_output=True, text=True, timeout=300, env=env)
+        if r.returncode != 0:
+            return {"error": f"rc {r.returncode}: {r.stderr[-300:]}"}
+        out = {}
+        for line in r.stdout.strip().splitlines():
+            k, v = line.split()
+            out[k + "_us"] = float(v)
+        return out
 
 
 def reduce_max_over_ranks(x: float, dist, device) -> float:
@@ -733,7 +797,8 @@ def run_native(args):
                 if name == args.workload:
                     continue
                 od = make_config(name)
-                ores = time_workload(od, device, max(10, min(args.steps, 50)), 3)
+                ores = time_workload(od, device, max(10, min(args.steps, 50)), 3, soak_s=0.5,
+                                     sampler=ClockSampler(local))
                 others[name] = {k: (round(v, 4) if isinstance(v, float) else v)
                                 for k, v in summarise(od, ores, peaks).items()}
                 del od
@@ -766,6 +831,24 @@ def run_native(args):
         "tensor_frac": w["flops"] / attn_s / 1e12 / peaks["bf16_tflops"],
         "note": "decode at H=128 does 242 flop per KV byte, just under the ridge; both fractions are reported",
     }
+    rooflines_other = {}
+    for name in ("mixed_prefill", "spec_shared_prefix"):
+        o = others.get(name)
+        if not o:
+            continue
+        achieved = o["flops"] / (o["attn_kernel_us"] * 1e-6) / 1e12
+        rooflines_other[name] = {
+            "bound": "tensor", "kernel": "mla_attn_kernel", "achieved": achieved,
+            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+            "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+            "peak_sustained": peaks["bf16_tflops_sustained"],
+            "traffic": kernel_traffic(name),
+            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json bf16_tflops burst; bf16_tflops_sustained beside)"
+                           if peak_kind == "measured" else "fallback",
+            "algorithmic_flops_per_launch": o["flops"], "kernel_us": o["attn_kernel_us"],
+            "step_us": o["us_per_step"],
+            "note": "2176 flop per visible (query row x head x key); kernel and step from the same timed steps",
+        }
     line = {
         "metric": METRIC,
         "value": value,
@@ -779,17 +862,18 @@ def run_native(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": f"{args.workload}: {d.description}", "parallelism": f"replicas x{world}",
-                   "l2": f"inputs rotated over {res['n_copies']} HBM copies ({input_bytes(d) / 1e6:.0f} MB each), "
-                         f"never L2-resident between steps",
-                   "kv_bytes_per_step": w["kv_bytes"], "flops_per_step": w["flops"]},
+        "config": config_of(args.workload, d),
+        "parallelism": f"replicas x{world}",
+        "l2_detail": f"inputs rotated over {res['n_copies']} HBM copies ({input_bytes(d) / 1e6:.0f} MB each)",
         "roofline": roofline,
+        "rooflines_other": rooflines_other,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": res["launches"],
         "clocks": res["clocks"],
         "tflops": summ["tflops"],
         "frac_tensor": summ["frac_tensor"],
+        "us_per_step_plain": summ["us_per_step_plain"],
         "others": others,
         "next_rows": next_rows,
     }

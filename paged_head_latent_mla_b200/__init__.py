@@ -116,8 +116,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             f"CUDA library {path} is missing: build it with "
             "`python -m paged_head_latent_mla_b200._build` (there is no fallback)")
     lib = ctypes.CDLL(path)
-    i32p = ctypes.POINTER(ctypes.c_int32)
     vp = ctypes.c_void_p
+    i32p = vp  # host int32 tables and out-arrays travel as addresses (see _ptr)
     lib.mla_supports.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
     lib.mla_supports.restype = ctypes.c_int
     lib.mla_plan.argtypes = [ctypes.POINTER(_Dims), ctypes.c_int32, i32p, i32p, i32p, i32p, ctypes.c_int32, vp,
@@ -161,6 +161,8 @@ mla_status_string = status_string
 
 
 def _i32(x) -> np.ndarray:
+    if type(x) is np.ndarray and x.dtype == np.int32 and x.flags.c_contiguous:
+        return x  # already what the library reads
     try:
         import torch
 
@@ -173,8 +175,9 @@ def _i32(x) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(x, dtype=np.int32))
 
 
-def _ptr(a: np.ndarray):
-    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+def _ptr(a: np.ndarray) -> int:
+    """Address of a host int32 array's data, for the table arguments (declared void*)."""
+    return a.ctypes.data
 
 
 def mla_supports(kv_lora_rank: int, rope_dim: int, num_heads: int, page_size: int) -> bool:
