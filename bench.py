@@ -339,6 +339,7 @@ def time_workload(d, device, steps, warmup, dist=None, soak_s=0.0, sampler=None,
     torch.cuda.synchronize(device)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    e2 = torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(steps):
         tstep()
@@ -346,16 +347,17 @@ def time_workload(d, device, steps, warmup, dist=None, soak_s=0.0, sampler=None,
     torch.cuda.synchronize(device)
     if dist is not None:
         dist.barrier()
-    clocks = sampler.stop() if sampler is not None else None
-    ms = e0.elapsed_time(e1)
-    attn_ms, merge_ms = M.mla_plan_kernel_times(tplan, capacity=min(steps, 256))
-    # the product path without events between its launches, same steps, right after
-    e0.record()
+    # The product path without events between its launches, the same steps, enqueued
+    # at once so that it runs under the same (power-capped) clocks; a pause here would
+    # let the clocks recover and flatter it.
     for _ in range(steps):
         pstep()
-    e1.record()
+    e2.record()
     torch.cuda.synchronize(device)
-    ms_plain = e0.elapsed_time(e1)
+    clocks = sampler.stop() if sampler is not None else None
+    ms = e0.elapsed_time(e1)
+    ms_plain = e1.elapsed_time(e2)
+    attn_ms, merge_ms = M.mla_plan_kernel_times(tplan, capacity=min(steps, 256))
     for pl in (plan, tplan):
         st = M.mla_plan_check(pl)
         if st != 0:
@@ -671,15 +673,26 @@ def measure_next_rows(device, peaks):
             fn(i)
         return (time.perf_counter() - t0) / n * 1e6
 
-    reuse_us = host_us(lambda i: M.mla_plan_update(plan, *tabs[0]))
-    replan_us = host_us(lambda i: M.mla_plan_update(plan, *tabs[i % 2]))
+    sid = torch.cuda.current_stream(device).cuda_stream  # given once, as a serving loop would
+    reuse_us = host_us(lambda i: M.mla_plan_update(plan, *tabs[0], stream=sid))
+    replan_us = host_us(lambda i: M.mla_plan_update(plan, *tabs[i % 2], stream=sid))
 
-    def fresh(i):
-        p = M.mla_plan(*tabs[i % 2], num_heads=d.num_heads, page_size=d.page_size,
-                       num_pages=max(d.num_pages, d2.num_pages), sm_scale=d.sm_scale, causal=d.causal)
-        p.destroy()
-
-    fresh_us = host_us(fresh)
+    # fresh plans, each destroyed two steps later (as a pipelined serving loop retires
+    # them); only the mla_plan calls are timed
+    live, spent = [], 0.0
+    for i in range(103):
+        t0 = time.perf_counter()
+        pl = M.mla_plan(*tabs[i % 2], num_heads=d.num_heads, page_size=d.page_size,
+                        num_pages=max(d.num_pages, d2.num_pages), sm_scale=d.sm_scale, causal=d.causal,
+                        stream=sid)
+        if i >= 3:
+            spent += time.perf_counter() - t0
+        live.append(pl)
+        if len(live) > 2:
+            live.pop(0).destroy()
+    for pl in live:
+        pl.destroy()
+    fresh_us = spent / 100 * 1e6
     torch.cuda.synchronize(device)
     plan.destroy()
     res["plan_reuse_decode_b64"] = {"unchanged_update_us": reuse_us, "changed_update_us": replan_us,

@@ -146,6 +146,49 @@ void pool_give(int kind, int device, void* ptr, size_t cap) {
   }
 }
 
+// The plan's events (last run, uploads) come from a per-device list as well: creating
+// and destroying them costs microseconds of host time on every plan.  At most
+// kEventKeep events per device are kept.
+struct PooledEvent {
+  cudaEvent_t ev;
+  int device;
+};
+std::vector<PooledEvent>* g_events = new std::vector<PooledEvent>();  // never destroyed
+constexpr int kEventKeep = 32;
+
+cudaEvent_t event_take(int device) {
+  {
+    std::lock_guard<std::mutex> lock(g_pool_mutex);
+    for (size_t i = g_events->size(); i-- > 0;)
+      if ((*g_events)[i].device == device) {
+        const cudaEvent_t e = (*g_events)[i].ev;
+        g_events->erase(g_events->begin() + static_cast<std::ptrdiff_t>(i));
+        return e;
+      }
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return e;
+}
+
+// The event must have completed (the plan was quiesced).
+void event_give(int device, cudaEvent_t e) {
+  if (!e) return;
+  {
+    std::lock_guard<std::mutex> lock(g_pool_mutex);
+    int n = 0;
+    for (const PooledEvent& x : *g_events) n += x.device == device;
+    if (n < kEventKeep) {
+      g_events->push_back(PooledEvent{e, device});
+      return;
+    }
+  }
+  cudaEventDestroy(e);
+}
+
 // Wait until no launch or upload of the plan can still be reading its buffers.
 void quiesce(mla_plan_s* p) {
   if (p->captured) {
@@ -163,9 +206,8 @@ void free_plan(mla_plan_s* p) {
   if (!p) return;
   if (!p->host_only) {
     quiesce(p);
-    if (p->ev_last) cudaEventDestroy(p->ev_last);
-    for (int i = 0; i < 2; ++i)
-      if (p->ev_upload[i]) cudaEventDestroy(p->ev_upload[i]);
+    event_give(p->device, p->ev_last);
+    for (int i = 0; i < 2; ++i) event_give(p->device, p->ev_upload[i]);
     if (p->ring) {
       for (int i = 0; i < 3 * mla_plan_s::kRing; ++i)
         if (p->ring[i]) cudaEventDestroy(p->ring[i]);
@@ -278,10 +320,7 @@ mla_status upload(mla_plan_s* p, const int32_t* kv_indices, int64_t n_idx, cudaS
       return MLA_ERR_OUT_OF_MEMORY;
     }
   }
-  if (!p->ev_upload[k] && cudaEventCreateWithFlags(&p->ev_upload[k], cudaEventDisableTiming) != cudaSuccess) {
-    cudaGetLastError();
-    return MLA_ERR_CUDA;
-  }
+  if (!p->ev_upload[k] && !(p->ev_upload[k] = event_take(p->device))) return MLA_ERR_CUDA;
   const PlanLayout& L = p->layout;
   uint8_t* h = static_cast<uint8_t*>(p->h_staging[k]);
   std::memset(h + p->sz.off_work, 0, p->sz.off_refs - p->sz.off_work);  // empty work and merge slots
@@ -492,8 +531,7 @@ mla_status mla_plan(const mla_dims* dims, int32_t batch, const int32_t* qo_indpt
     for (int i = 0; i < 3 * mla_plan_s::kRing; ++i)
       if (cudaEventCreate(&p->ring[i]) != cudaSuccess) { cudaGetLastError(); free_plan(p); return MLA_ERR_CUDA; }
   }
-  if (cudaEventCreateWithFlags(&p->ev_last, cudaEventDisableTiming) != cudaSuccess) {
-    cudaGetLastError();
+  if (!(p->ev_last = event_take(p->device))) {
     free_plan(p);
     return MLA_ERR_CUDA;
   }

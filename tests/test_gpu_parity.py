@@ -282,3 +282,58 @@ def test_pooled_plan_buffers_reused_across_shapes():
     check(2, ob, lb)
     a.destroy()
     b.destroy()
+
+
+def _with_common_offset(d, q_shift, k_shift, seed):
+    """The same step with a shared direction added to every query and every key: each
+    score gains about q_shift * k_shift * 576 * sm_scale, the same for every key of a
+    row up to the keys' own spread, so the scores sit far from zero while their
+    differences stay those of the random parts."""
+    g = torch.Generator().manual_seed(seed)
+    u = torch.randn(576, generator=g)
+    u = u / u.norm()
+    d.q_nope = (d.q_nope.float() + q_shift * u[:512]).to(torch.bfloat16)
+    d.q_pe = (d.q_pe.float() + q_shift * u[512:]).to(torch.bfloat16)
+    d.cache = (d.cache.float() + k_shift * u).to(torch.bfloat16)
+    return d
+
+
+def test_scores_far_from_zero():
+    """Scores near +300 natural units, with the usual spread between keys.  The pair of
+    CTAs exchanges its partial scores as 16-bit offsets below a per-row anchor, so the
+    precision must not depend on the scores' distance from zero."""
+    d = make_custom([1, 4, 1], [900, 300, 2000], 128, 64, seed=37)
+    d = _with_common_offset(d, 60.0, 60.0, seed=38)  # 60 * 60 * 0.072 = 260 in the score
+    out, lse, _, _ = gpu_run(d)
+    compare(d, out, lse)
+    assert np.nanmin(lse) > 200  # the offset is really there
+
+
+def test_opposite_half_partials():
+    """Keys whose large scores come from opposite halves of the latent width: key A's
+    from ckv columns [0, 256) and kpe [0, 32), key B's from ckv [256, 512) and kpe
+    [32, 64), the two halves that the two CTAs of a pair hold.  Each CTA then sees one
+    key's partial far above the other's (about 150 natural units apart), while their
+    full scores are equal.  The partials travel between the CTAs in a 16-bit code
+    whose step follows each row's span, so both keys keep equal weight, as the oracle
+    has them, alongside keys with a wide random spread of scores from the rope part."""
+    d = make_custom([1, 1, 3], [40, 100, 130], 16, 16, seed=41)
+    g = torch.Generator().manual_seed(42)
+    c = d.cache.float()
+    c[..., 512:] *= torch.exp(torch.randn((d.num_pages, d.page_size, 1), generator=g) * 1.5) * 4.0
+    qn, qp = d.q_nope.float(), d.q_pe.float()
+    qv = torch.cat([qn[0, 0], qp[0, 0]])  # row 0's query (all its heads share it)
+    qn[0, :] = qv[:512]
+    qp[0, :] = qv[512:]
+    half0 = torch.zeros(576, dtype=torch.bool)
+    half0[:256] = True
+    half0[512:544] = True
+    target = 150.0 / d.sm_scale  # score of 150 natural units
+    kvp, idx = d.kv_indptr.numpy(), d.kv_indices.numpy()
+    for key, mask in ((5, half0), (27, ~half0)):
+        page, slot = int(idx[kvp[0] + key // d.page_size]), key % d.page_size
+        v = torch.where(mask, qv, torch.zeros_like(qv))
+        c[page, slot] = v * (target / float(v @ v))
+    d.cache, d.q_nope, d.q_pe = c.to(torch.bfloat16), qn.to(torch.bfloat16), qp.to(torch.bfloat16)
+    out, lse, _, _ = gpu_run(d)
+    compare(d, out, lse)
