@@ -20,14 +20,11 @@
 //    every key, so every cache byte crosses HBM once.
 //  * Per 64-key tile: each CTA computes a partial S = Q_half . K_half^T (tcgen05,
 //    M=128, N=64, K=288) into TMEM; the exchange warps push it to the peer over DSMEM
-//    (st.async completing on the peer's mbarrier) as 16-bit fixed-point offsets below
-//    a per-row anchor with a per-row power-of-two step (16.5 KB a tile instead of 32 KB
-//    of fp32; see the encoding constants for the error), into one of two slots; the softmax
-//    warps add the decoded peer partial to their own fp32 one, apply mask and online
-//    softmax (log2 domain, lazy rescale), and store P as bf16 into TMEM.  Each CTA
-//    normalises its own half of O by its own running sum, so the two halves need not
-//    hold bit-identical scores.  Then O_half += P . V_half (tcgen05, A = P from TMEM,
-//    B = the ckv columns of the same shared-memory tile read MN-major, N = 256).
+//    (st.async completing on the peer's mbarrier); the softmax warps add the peer's
+//    partial (fp32 addition commutes, so both CTAs hold bit-identical S), apply mask
+//    and online softmax (log2 domain, lazy rescale), and store P as bf16 into TMEM.
+//    Then O_half += P . V_half (tcgen05, A = P from TMEM, B = the ckv columns of the
+//    same shared-memory tile read MN-major, N = 256).
 //  * Roles (11 warps): warps 0..3 softmax and epilogue, 4..7 exchange (one per TMEM
 //    lane quarter in each group), 8 TMA producer, 9 QK issuer (one thread; also TMEM
 //    allocation and zeroing of key rows past the row's end), 10 PV issuer.
@@ -57,7 +54,7 @@ namespace attn {
 #define MLA_KV_STAGES 4
 #endif
 #ifndef MLA_X_SLOTS
-#define MLA_X_SLOTS 2
+#define MLA_X_SLOTS 1
 #endif
 constexpr int kStages = MLA_KV_STAGES;  // KV ring depth
 constexpr int kXSlots = MLA_X_SLOTS;    // exchange buffers (1 or 2)
@@ -79,12 +76,7 @@ constexpr uint32_t kKV = 49152;            // kStages stages
 constexpr uint32_t kStageBytes = 36864;    //   4 chunks x [64 keys x 128 B] + [64 x 64 B]
 constexpr uint32_t kStageKpe = 32768;
 constexpr uint32_t kX = kKV + kStages * kStageBytes;  // the peer's partial scores
-// One exchange slot: the peer's 128 x 64 partial scores as 16-bit fixed-point offsets
-// below a per-row anchor (4 quarters x 8 chunks x 32 lanes x 16 B), then the 128 anchors.
-constexpr uint32_t kXQuarterBytes = 8 * 32 * 16;
-constexpr uint32_t kXAnchor = 4 * kXQuarterBytes;
-constexpr uint32_t kXSlotBytes = kXAnchor + 128 * 4;
-constexpr uint32_t kXQuarterTx = kXQuarterBytes + 32 * 4;  // bytes one quarter's barrier counts
+constexpr uint32_t kXSlotBytes = 128 * 64 * 4;       // 4 quarters x 16 chunks x 32 lanes x 16 B
 constexpr uint32_t kBar = kX + kXSlots * kXSlotBytes;
 constexpr uint32_t kMisc = kBar + 512;
 constexpr uint32_t kSmemUsed = kMisc + 64;
@@ -117,21 +109,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kQBytes = kQSmemChunks * 16384;
 constexpr float kNegInf = -__builtin_huge_valf();
 
-// Exchange encoding (block floating point per row and tile).  With v_j = s_j * scale_log2
-// the log2-domain partial scores of a row over the tile's keys that hold cache rows,
-// the sender picks the step e = the smallest power of two with e >= (max v - min v) /
-// 65534 and e >= |max v| / 2^22, the anchor R = round(max v / e), and sends
-// u_j = round(R - v_j / e), an integer in [0, 65535] (clamped only for keys past the
-// row's end, which the receiver masks), plus one float per row, cr = (R + 1.5 * 2^23) * e.
-// The receiver reads e from cr's exponent (R + 1.5 * 2^23 lies in [2^23, 2^24)) and
-// takes cr - (1.5 * 2^23 + u_j) * e = (R - u_j) * e, exactly, as the peer's part.  The
-// error is at most e / 2: 2^-10 log2 units or less whenever the row's partials span at
-// most 64 log2 units and lie within 2^13 of zero, and never more than 1/65534 of
-// their span plus 2^-22 of their size.  Rounding uses the float magic number
-// 1.5 * 2^23, whose unit in the last place is 1.
-constexpr float kXMagic = 12582912.0f;              // 1.5 * 2^23: bits 0x4B400000
-constexpr float kXMagicTop = 12582912.0f + 65535.0f;
-
 // Error sites (bits 8.. of the status word) for diagnosis.
 enum : int32_t {
   kSiteProducer = 1,
@@ -154,12 +131,11 @@ __device__ __forceinline__ void record_error(int32_t* status, int32_t site) {
 }  // namespace attn
 
 // Pipeline per 64-key tile j (phases of every two-buffer barrier are j >> 1):
-//   producer : KV(j) -> stage j % 4                        (after PV(j - 4) freed it)
+//   producer : KV(j) -> stage j % 3                        (after PV(j - 3) freed it)
 //   QK warp  : QK(j) -> S[j % 2], as soon as KV(j) landed and S(j - 2) was read
-//   exchange : S(j) partial, encoded -> peer's slot j % 2 over DSMEM (st.async, completes
-//              the peer's x_full), once the peer has drained tile j - 2 from that slot
+//   exchange : S(j) partial -> peer over DSMEM (st.async, completes the peer's x_full)
 //   softmax  : S(j) = ours + peer's; mask, online softmax, P(j) -> P[j % 2]
-//   PV warp  : PV(j): O += P[j % 2] . V(stage j % 4), as soon as P(j) is written
+//   PV warp  : PV(j): O += P[j % 2] . V(stage j % 3), as soon as P(j) is written
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     mla_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                     const __grid_constant__ CUtensorMap tm_kpe, const AttnParams p) {
@@ -372,61 +348,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     }
   } else if (warp >= kWarpExchange0) {
     // ------------------------------------------------------------------ score exchange
-    // Partial S(j) (our 288 of the 576 contraction columns) goes to the peer in the
-    // 16-bit encoding above, laid out chunk-major per lane quarter: 16-byte chunk c of
-    // row (32q + lane) sits at q * 4 KB + (c * 32 + lane) * 16, so one warp store covers
-    // 512 contiguous bytes; the row's anchor follows in the slot's anchor area.
+    // Partial S(j) (our 288 of the 576 contraction columns) goes to the peer, laid out
+    // chunk-major per lane quarter: 16-byte chunk c of row (32q + lane) sits at
+    // q * 8 KB + (c * 32 + lane) * 16, so one warp store covers 512 contiguous bytes.
     const int q = warp & 3;
     const uint32_t trow = tmem + (static_cast<uint32_t>(32 * q) << 16);
-    const uint32_t xq_peer = map_to_cta(sb + kX + q * kXQuarterBytes + lane * 16, peer);
-    const uint32_t xa_peer = map_to_cta(sb + kX + kXAnchor + (32 * q + lane) * 4, peer);
+    const uint32_t xq_peer = map_to_cta(sb + kX + q * 8192 + lane * 16, peer);
     const uint32_t xfull_peer = map_to_cta(bar(bXFull + q), peer);
-    const float sc = p.scale_log2;
     for (int j = 0; j < ntiles; ++j) {
       const int b2 = j & 1;
       if (!wait_warp(bar(bSFull + b2), (j >> 1) & 1, kSiteExchange, false)) break;
       tc_fence_after();
       uint32_t sr[64];
-      tmem_ld64(trow + kColS + 64 * b2, sr);
+      tmem_ld32(trow + kColS + 64 * b2, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(trow + kColS + 64 * b2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(bSEmpty + b2));
-      // the row's span over the tile's keys that hold cache rows (keys past the row's
-      // end may hold anything), then its step, anchor and codes (encoding above)
-      const int nkv = min(kTileN, w.kv_len - (w.key_begin + kTileN * j));
-      float vmax = kNegInf, vmin = -kNegInf;
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float v = __uint_as_float(sr[c]);
-        vmax = (c < nkv) ? fmaxf(vmax, v) : vmax;
-        vmin = (c < nkv) ? fminf(vmin, v) : vmin;
-      }
-      const float amax = vmax * sc;
-      float x = fmaxf(fmaxf((vmax - vmin) * sc * (1.0f / 65534.0f), fabsf(amax) * (1.0f / 4194304.0f)),
-                      9.3132257e-10f);  // at least 2^-30
-      if (!(x <= 1073741824.0f)) x = 1.0f;  // non-finite partials: any step will do
-      const uint32_t e_bits = (__float_as_uint(x) + 0x007FFFFFu) & 0x7F800000u;  // next power of 2
-      const float inv_e = __uint_as_float((254u << 23) - e_bits);
-      float R = rintf(amax * inv_e);
-      if (!(fabsf(R) <= 4194304.0f)) R = 0.f;
-      const float C = R + kXMagic, qs = sc * inv_e;
-      uint32_t pk[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float f0 = fminf(fmaxf(fmaf(__uint_as_float(sr[2 * c]), -qs, C), kXMagic), kXMagicTop);
-        const float f1 = fminf(fmaxf(fmaf(__uint_as_float(sr[2 * c + 1]), -qs, C), kXMagic), kXMagicTop);
-        pk[c] = prmt(__float_as_uint(f0), __float_as_uint(f1), 0x5410u);  // the two low halves
-      }
-      const float cr = C * __uint_as_float(e_bits);
       // the peer must have drained our slot (it held tile j - kXSlots)
       const int xs = j % kXSlots, xph = j / kXSlots;
       if (j >= kXSlots && !wait_warp(bar(bXEmpty + 4 * xs + q), (xph - 1) & 1, kSiteExchange, true)) break;
       const uint32_t dst = xq_peer + xs * kXSlotBytes;
       const uint32_t xbar = xfull_peer + 8u * (4 * xs);
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        st_async_v4(dst + c * 512, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3], xbar);
-      st_async_b32(xa_peer + xs * kXSlotBytes, __float_as_uint(cr), xbar);
+      for (int c = 0; c < 16; ++c)
+        st_async_v4(dst + c * 512, sr[4 * c], sr[4 * c + 1], sr[4 * c + 2], sr[4 * c + 3], xbar);
     }
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
@@ -437,8 +384,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     vis = max(0, min(vis, w.kv_len));
     if (r >= w.n_rows) vis = 0;
     const int lim = min(vis, w.key_end);  // keys < lim are visible in this chunk
-    const uint8_t* xq_ptr = smem + kX + q * kXQuarterBytes + lane * 16;
-    const float* xa_ptr = reinterpret_cast<const float*>(smem + kX + kXAnchor) + r;
+    const float* xq_ptr = reinterpret_cast<const float*>(smem + kX + q * 8192 + lane * 16);
     const float scale = p.scale_log2;  // > 0 (the planner rejects other scales)
     float m_run = kNegInf, l_run = 0.f;
     bool ok = true;
@@ -486,32 +432,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       if (!(ok = wait_warp(bar(bSFull + b2), (j >> 1) & 1, kSiteSoftS, false))) break;
       const int xsl = j % kXSlots, xph = j / kXSlots;
       const uint32_t xfull = bar(bXFull + 4 * xsl + q);
-      if (lane == 0) mbar_arrive_expect_tx(xfull, kXQuarterTx);
+      if (lane == 0) mbar_arrive_expect_tx(xfull, 8192);
       tc_fence_after();
       uint32_t sr[64];
-      tmem_ld64(trow + kColS + 64 * b2, sr);
+      tmem_ld32(trow + kColS + 64 * b2, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(trow + kColS + 64 * b2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(bSEmpty + b2));
       if (!(ok = wait_warp(xfull, xph & 1, kSiteSoftX, true))) break;
-      // --- S(j) in the log2 domain: our fp32 partial times the scale, plus the peer's
-      // decoded part (R - u) * e.  u arrives as the low 16 bits of a float whose high
-      // bits are those of kXMagic, so that float is kXMagic + u, and cr - f * e is exact.
-      const uint8_t* xs = xq_ptr + xsl * kXSlotBytes;
-      const float cr = xa_ptr[xsl * (kXSlotBytes / 4)];
-      const float xe = __uint_as_float((__float_as_uint(cr) & 0x7F800000u) - (23u << 23));
+      // --- raw S(j) = our partial + the peer's (fp32 addition commutes: the pair holds
+      // bit-identical scores)
+      const float* xs = xq_ptr + xsl * (kXSlotBytes / 4);
       float t[64];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 x = *reinterpret_cast<const uint4*>(xs + c * 512);
-        const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float lo = __uint_as_float(prmt(xw[k], 0x4B400000u, 0x7610u));
-          const float hi = __uint_as_float(prmt(xw[k], 0x4B400000u, 0x7632u));
-          t[8 * c + 2 * k] = fmaf(__uint_as_float(sr[8 * c + 2 * k]), scale, fmaf(lo, -xe, cr));
-          t[8 * c + 2 * k + 1] = fmaf(__uint_as_float(sr[8 * c + 2 * k + 1]), scale, fmaf(hi, -xe, cr));
-        }
+      for (int c = 0; c < 16; ++c) {
+        const float4 x = *reinterpret_cast<const float4*>(xs + c * 128);
+        t[4 * c + 0] = __uint_as_float(sr[4 * c + 0]) + x.x;
+        t[4 * c + 1] = __uint_as_float(sr[4 * c + 1]) + x.y;
+        t[4 * c + 2] = __uint_as_float(sr[4 * c + 2]) + x.z;
+        t[4 * c + 3] = __uint_as_float(sr[4 * c + 3]) + x.w;
       }
 
       // --- mask (partial tiles only), running max in the log2 domain, lazy rescale
@@ -527,14 +468,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       for (int c = 16; c < 64; c += 8)
 #pragma unroll
         for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], t[c + i]);
-      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      // Hand the slot back to the peer.  mt depends on every value loaded from the
-      // slot, and the vote needs every lane's mt, so all of this warp's loads have
+      const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      const float mt = mraw * scale;  // scale > 0 keeps the order; -inf stays -inf
+      // Hand the slot back to the peer.  mraw depends on every value loaded from the
+      // slot, and the vote needs every lane's mraw, so all of this warp's loads have
       // delivered their data before lane 0's arrive issues; the peer's next push cannot
       // overtake them.  (An arrive issued before the loads completed did let it; a
       // release-ordered arrive also works but costs a cluster-scope fence per tile.)
-      if (__any_sync(0xffffffffu, mt != p.nan_guard) && lane == 0)
+      if (__any_sync(0xffffffffu, mraw != p.nan_guard) && lane == 0)
         mbar_arrive_remote_relaxed(bar(bXEmpty + 4 * xsl + q), peer);
       // Keep the old reference max unless the new one exceeds it by more than 8 (a
       // factor of 256 in the weights); then rescale the running sum and output row.
@@ -570,8 +512,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        const float p0 = ex2_approx(t[2 * c] - msub);
-        const float p1 = ex2_approx(t[2 * c + 1] - msub);
+        const float p0 = ex2_approx(fmaf(t[2 * c], scale, -msub));
+        const float p1 = ex2_approx(fmaf(t[2 * c + 1], scale, -msub));
         pk[c] = pack_bf16x2(p0, p1);
         ls[c & 3] += p0 + p1;
       }
