@@ -10,6 +10,7 @@
 #include <limits>
 #include <mutex>
 #include <new>
+#include <utility>
 #include <vector>
 
 #include "mla_internal.h"
@@ -24,6 +25,7 @@ struct mla_plan_s {
   bool causal = true;
   mla_plan_options opts{};
   PlanLayout layout;
+  PlanLayout spare;  // the previous step's layout, kept so a re-plan reuses its capacity
   int device = -1;
   bool host_only = false;
   bool graph = false;     // fixed buffers and launch shapes (opts.graph_max_*)
@@ -559,12 +561,14 @@ mla_status mla_plan_update(mla_plan_t p, int32_t batch, const int32_t* qo_indptr
   if (!p->host_only) {
     if (check_device(p) != MLA_OK || stream_capturing(s)) return MLA_ERR_INVALID_ARGUMENT;
   }
-  PlanLayout L;
+  // The new layout is built in the spare one (whose vectors keep their capacity from
+  // earlier steps), then the two are swapped.
+  PlanLayout& L = p->spare;
   mla_status st = build_layout(request_of(p, batch, qo_indptr, kv_indptr, kv_indices, last_page_len), &L);
   if (st != MLA_OK) return st;
   const int64_t n_idx = batch > 0 ? kv_indptr[batch] : 0;
   if (p->host_only) {
-    p->layout = std::move(L);
+    std::swap(p->layout, p->spare);
     remember_tables(p, batch, qo_indptr, kv_indptr, kv_indices, last_page_len);
     return MLA_OK;
   }
@@ -576,11 +580,10 @@ mla_status mla_plan_update(mla_plan_t p, int32_t batch, const int32_t* qo_indptr
     p->sz = saved;
     return st;
   }
-  PlanLayout old = std::move(p->layout);
-  p->layout = std::move(L);
+  std::swap(p->layout, p->spare);
   st = upload(p, kv_indices, n_idx, s);
   if (st != MLA_OK) {
-    p->layout = std::move(old);
+    std::swap(p->layout, p->spare);  // the plan keeps describing its previous step
     return st;
   }
   remember_tables(p, batch, qo_indptr, kv_indptr, kv_indices, last_page_len);

@@ -11,9 +11,7 @@
 // the cascade option exploits by attending such a prefix once per group of rows.
 #include <algorithm>
 #include <cmath>
-#include <functional>
 #include <limits>
-#include <queue>
 
 #include "mla_internal.h"
 
@@ -219,15 +217,17 @@ bool fits(const std::vector<QTile>& tiles, int32_t n_out, int32_t chunk, const P
 
 // Longest-processing-time-first makespan of the items a split size gives, over `units`
 // identical SM pairs, plus the merge pass (which reads every partial once, spread over
-// all units).  The costs are whole numbers no larger than `max_cost`, so they are sorted
-// by counting; the unit loads live in a binary min-heap.  Stops early (returning a value
-// >= `give_up`) once the makespan cannot end below `give_up`.
+// all units).  The costs are whole numbers no larger than `max_cost`, so the items are
+// sorted by counting; and since the least loaded unit's load never decreases while items
+// are placed, the units are kept as counts per load value with a pointer to the least
+// load that only moves forward.  Stops early (returning a value >= `give_up`) once the
+// makespan cannot end below `give_up`.
 double estimate(const std::vector<QTile>& tiles, int32_t chunk, int units, int32_t max_cost,
                 double give_up = std::numeric_limits<double>::infinity()) {
-  static thread_local std::vector<int32_t> count;  // items per cost
-  static thread_local std::vector<int64_t> load;   // unit loads (min-heap)
+  static thread_local std::vector<int32_t> count;   // items per cost
+  static thread_local std::vector<int32_t> at_load; // units per load value
   count.assign(static_cast<size_t>(max_cost) + 1, 0);
-  int64_t partials = 0;
+  int64_t partials = 0, total = 0;
   for (const QTile& t : tiles) {
     const int32_t n = pieces_for(t.ntiles, chunk);
     const bool part = n > 1 || t.must_merge;
@@ -236,33 +236,27 @@ double estimate(const std::vector<QTile>& tiles, int32_t chunk, int units, int32
     const int32_t q = t.ntiles / n, r = t.ntiles % n;
     if (r > 0) count[q + 1 + fixed] += r;
     count[q + fixed] += n - r;
+    total += int64_t(t.ntiles) + int64_t(n) * fixed;
     if (part) partials += n;
   }
   const double merge = kSplitCost * double(partials) / units;
   const double limit = give_up - merge;
-  // The least loaded unit takes the next longest item: its load grows in place at the
-  // root of the heap, which is then sifted down.
-  load.assign(static_cast<size_t>(units), 0);  // all zero: already a heap
-  int64_t* h = load.data();
-  const int m = units;
-  int64_t worst = 0;
+  // every load stays below the makespan, which stays below min(total, limit) + max_cost
+  int64_t top = total;
+  if (limit < double(top)) top = std::max<int64_t>(0, static_cast<int64_t>(limit) + 1);
+  at_load.assign(static_cast<size_t>(top + max_cost) + 2, 0);
+  at_load[0] = units;
+  int64_t least = 0, worst = 0;
   for (int32_t cost = max_cost; cost >= 0; --cost) {
     for (int32_t k = count[cost]; k > 0; --k) {
-      const int64_t l = h[0] + cost;
+      while (at_load[least] == 0) ++least;
+      const int64_t l = least + cost;
+      --at_load[least];
+      ++at_load[l];
       if (l > worst) {
         worst = l;
         if (double(worst) >= limit) return double(worst) + merge;
       }
-      int i = 0;
-      for (;;) {
-        const int a = 2 * i + 1, b = a + 1;
-        if (a >= m) break;
-        const int c = (b < m && h[b] < h[a]) ? b : a;
-        if (h[c] >= l) break;
-        h[i] = h[c];
-        i = c;
-      }
-      h[i] = l;
     }
   }
   return double(worst) + merge;
@@ -300,8 +294,16 @@ mla_status build_layout(const PlanRequest& req, PlanLayout* out) {
   const int64_t n_idx = kv_indptr[batch];
   if (T * H > std::numeric_limits<int32_t>::max() - kTileM) return MLA_ERR_INVALID_ARGUMENT;
   if (n_idx > 0 && !kv_indices) return MLA_ERR_INVALID_ARGUMENT;
-  for (int64_t i = 0; i < n_idx; ++i)
-    if (kv_indices[i] < 0 || kv_indices[i] >= d.num_pages) return MLA_ERR_INVALID_ARGUMENT;
+  {
+    // every page id in [0, num_pages): one pass for the smallest and largest id
+    int32_t lo = 0, hi = 0;
+    if (n_idx > 0) lo = hi = kv_indices[0];
+    for (int64_t i = 0; i < n_idx; ++i) {
+      lo = std::min(lo, kv_indices[i]);
+      hi = std::max(hi, kv_indices[i]);
+    }
+    if (lo < 0 || hi >= d.num_pages) return MLA_ERR_INVALID_ARGUMENT;
+  }
 
   // --- per-row key counts (k_b from the tables; c_b = k_b - q_b attended if context-only)
   // Working arrays live in per-thread scratch that keeps its capacity from call to call,
