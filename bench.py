@@ -469,6 +469,51 @@ def time_e2e(d, device, steps, warmup):
     return ms, h2d[0], d2h
 
 
+def time_e2e_cpp(d, steps, warmup):
+    """The same end-to-end loop as time_e2e, written as a C++ client of the C ABI
+    (tests/c/e2e_driver.cpp): per step mla_plan from host tables, H2D of the queries from
+    pinned memory, mla_run, D2H of the result to pinned memory, pipelined two deep on
+    three streams, each plan retired two steps later.  Returns (ms/step, h2d bytes, d2h
+    bytes), or a dict with an error when no compiler is at hand or the run fails."""
+    import shutil
+
+    import numpy as np
+    import torch
+
+    cxx = shutil.which("g++") or shutil.which("c++")
+    if cxx is None:
+        return {"error": "no C++ compiler"}
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    pkg = os.path.join(ROOT, "paged_head_latent_mla_b200")
+    with tempfile.TemporaryDirectory() as tmp:
+        exe = os.path.join(tmp, "e2e_driver")
+        r = subprocess.run([cxx, "-O2", "-std=c++17", "-I", os.path.join(ROOT, "include"), "-I",
+                            os.path.join(cuda, "include"), os.path.join(ROOT, "tests", "c", "e2e_driver.cpp"),
+                            "-L", pkg, "-l:libmla_b200.so", "-L", os.path.join(cuda, "lib64"), "-lcudart",
+                            "-Wl,-rpath," + pkg + ":" + os.path.join(cuda, "lib64"), "-o", exe],
+                           capture_output=True, text=True)
+        if r.returncode != 0:
+            return {"error": r.stderr[-300:]}
+        hdr = np.array([d.num_heads, d.page_size, d.num_pages, d.batch, 1 if d.causal else 0], np.int32)
+        with open(os.path.join(tmp, "tables"), "wb") as f:
+            for a in (hdr, d.qo_indptr.numpy(), d.kv_indptr.numpy(), d.kv_indices.numpy(),
+                      d.last_page_len.numpy()):
+                f.write(np.ascontiguousarray(a, dtype=np.int32).tobytes())
+        for name, t in (("q_nope.bin", d.q_nope), ("q_pe.bin", d.q_pe), ("cache.bin", d.cache)):
+            with open(os.path.join(tmp, name), "wb") as f:
+                f.write(t.contiguous().view(torch.int16).numpy().tobytes())
+        with open(os.path.join(tmp, "lse"), "wb") as f:
+            f.write(np.array([1 if d.return_lse else 0], np.int32).tobytes())
+        r = subprocess.run([exe, tmp, str(steps), str(warmup), repr(float(d.sm_scale))], capture_output=True,
+                           text=True, timeout=300)
+        if r.returncode != 0:
+            return {"error": f"rc {r.returncode}: {r.stderr[-300:]}"}
+        out = dict(line.split() for line in r.stdout.strip().splitlines())
+        if int(out["status"]) != 0:
+            return {"error": f"device status {out['status']}"}
+        return float(out["ms_per_step"]), int(out["h2d_bytes_per_step"]), int(out["d2h_bytes_per_step"])
+
+
 def summarise(d, res, peaks):
     w = work_of(d)
     s = res["ms_per_step"] * 1e-3
@@ -793,14 +838,27 @@ def run_native(args):
 
     e2e = None
     if not args.no_e2e:
-        e2e_ms, h2d, d2h = time_e2e(d, device, max(5, min(args.steps, 30)), 3)
-        e2e_ms = reduce_max_over_ranks(e2e_ms, dist, device)
-        e2e = {"value": job_throughput(w["kv_bytes"], world, e2e_ms), "unit": "GB/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms,
-               "includes": "per step: mla_plan from host tables + H2D of queries from pinned memory + mla_run "
-                           "+ D2H of out/lse to pinned memory; steps pipelined two deep on separate copy and "
-                           "compute streams; each plan's status word read two steps later; CUDA events from "
-                           "before the first plan to the last result on the host"}
+        e2e_steps = max(5, min(args.steps, 30))
+        py_ms, py_h2d, py_d2h = time_e2e(d, device, e2e_steps, 3)
+        py_ms = reduce_max_over_ranks(py_ms, dist, device)
+        loop = ("per step: mla_plan from host tables + H2D of queries from pinned memory + mla_run + D2H of "
+                "out/lse to pinned memory; steps pipelined two deep on separate copy and compute streams; each "
+                "plan's status word read two steps later; CUDA events from before the first plan to the last "
+                "result on the host")
+        e2e_python = {"value": job_throughput(w["kv_bytes"], world, py_ms), "unit": "GB/s",
+                      "h2d_bytes_per_step": int(py_h2d), "d2h_bytes_per_step": int(py_d2h), "ms_per_step": py_ms,
+                      "client": "Python binding (paged_head_latent_mla_b200)"}
+        cpp = time_e2e_cpp(d, e2e_steps, 3)
+        # every rank takes the same collective steps: a failed C++ run reports inf
+        cpp_ms = reduce_max_over_ranks(cpp[0] if isinstance(cpp, tuple) else float("inf"), dist, device)
+        if isinstance(cpp, tuple) and cpp_ms != float("inf"):
+            e2e = {"value": job_throughput(w["kv_bytes"], world, cpp_ms), "unit": "GB/s",
+                   "h2d_bytes_per_step": cpp[1], "d2h_bytes_per_step": cpp[2], "ms_per_step": cpp_ms,
+                   "client": "C++ through the C ABI (tests/c/e2e_driver.cpp)", "includes": loop,
+                   "python": e2e_python}
+        else:
+            e2e = dict(e2e_python, includes=loop,
+                       cpp_error=cpp.get("error") if isinstance(cpp, dict) else "failed on another rank")
 
     others = {}
     cpu = None

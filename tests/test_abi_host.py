@@ -232,3 +232,29 @@ def test_plan_timer_cpp_client(tmp_path):
     assert all(v > 0 for v in got.values())
     assert got["update_same"] < got["update_changed"]  # an unchanged step is only compared
     print("host-only planning, decode_b64 (us):", got)
+
+
+def test_e2e_cpp_client_builds(tmp_path):
+    """The C++ end-to-end client that the benchmark times on the GPU (plan, upload, run,
+    download, pipelined two deep through the C ABI) compiles warning-free against
+    include/mla.h and the CUDA runtime and links the library; without a GPU it is only
+    built, and it refuses a missing argument list."""
+    import shutil
+    import subprocess
+
+    cxx = shutil.which("g++") or shutil.which("c++")
+    if cxx is None:
+        pytest.skip("no C++ compiler")
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    if not os.path.exists(os.path.join(cuda, "include", "cuda_runtime.h")):
+        pytest.skip("no CUDA runtime headers")
+    lib_dir = os.path.dirname(M.LIB_PATH)
+    exe = str(tmp_path / "e2e_driver")
+    r = subprocess.run([cxx, "-O2", "-std=c++17", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), "-I",
+                        os.path.join(cuda, "include"), os.path.join(ROOT, "tests", "c", "e2e_driver.cpp"), "-L",
+                        lib_dir, "-l:libmla_b200.so", "-L", os.path.join(cuda, "lib64"), "-lcudart",
+                        "-Wl,-rpath," + lib_dir + ":" + os.path.join(cuda, "lib64"), "-o", exe],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 2 and "usage" in r.stderr
