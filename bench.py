@@ -415,9 +415,12 @@ def time_e2e(d, device, steps, warmup):
 
     def one(i):
         b = bufs[i % 2]
+        # the plan's upload goes on the upload stream ahead of the queries (on the compute
+        # stream it would wait for step i-1's run, then queue behind step i+1's query copy
+        # in the copy engine); `uploaded` orders the run after both
         plan = M.mla_plan(d.qo_indptr, d.kv_indptr, d.kv_indices, d.last_page_len, num_heads=H,
                           page_size=d.page_size, num_pages=d.num_pages, sm_scale=d.sm_scale, causal=d.causal,
-                          stream=s_run.cuda_stream)
+                          stream=s_up.cuda_stream)
         info = M.mla_plan_get_info(plan)
         with torch.cuda.stream(s_up):
             s_up.wait_event(b["computed"])  # step i-2 has finished reading these buffers
@@ -448,12 +451,12 @@ def time_e2e(d, device, steps, warmup):
     while live:
         retire(live.pop(0))
     torch.cuda.synchronize(device)
-    # device clock: from an event the compute stream passes before the first step is
-    # planned to one the download stream passes after the last result reached the host
+    # device clock: from an event the upload stream passes before the first step's plan
+    # upload to one the download stream passes after the last result reached the host
     # (host planning time shows up as device idle time inside the span)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(s_run)
+    e0.record(s_up)
     for i in range(steps):
         one(i)
     for b in bufs:
@@ -841,8 +844,9 @@ def run_native(args):
         e2e_steps = max(5, min(args.steps, 30))
         py_ms, py_h2d, py_d2h = time_e2e(d, device, e2e_steps, 3)
         py_ms = reduce_max_over_ranks(py_ms, dist, device)
-        loop = ("per step: mla_plan from host tables + H2D of queries from pinned memory + mla_run + D2H of "
-                "out/lse to pinned memory; steps pipelined two deep on separate copy and compute streams; each "
+        loop = ("per step: mla_plan from host tables (its upload on the copy stream) + H2D of queries from pinned "
+                "memory + mla_run + D2H of out/lse to pinned memory; steps pipelined two deep on separate copy "
+                "and compute streams; each "
                 "plan's status word read two steps later; CUDA events from before the first plan to the last "
                 "result on the host")
         e2e_python = {"value": job_throughput(w["kv_bytes"], world, py_ms), "unit": "GB/s",

@@ -145,7 +145,9 @@ int mla_supports(int kv_lora_rank, int rope_dim, int num_heads, int page_size);
  *   last_page_len host int32 [batch]; in [1, page_size] for a row with pages, ignored
  *                 (any value in [0, page_size]) for a row without
  *   causal        0 or 1
- *   stream        cudaStream_t (may be NULL) for the plan's uploads
+ *   stream        cudaStream_t (may be NULL) for the plan's uploads; a run on another
+ *                 stream must be ordered after them by the caller (an event recorded
+ *                 on `stream` after this call, or after later work of `stream`)
  *   opts          NULL or knobs above
  *   out_plan      receives the plan
  * The library copies every host array; the caller may reuse them on return.  The plan
@@ -177,7 +179,10 @@ mla_status mla_run(mla_plan_t plan, const void* q_nope, const void* q_pe, const 
                    void* out, float* lse, void* stream);
 
 /* Wait for the plan's last run to finish and report (then clear) its device status
- * word: MLA_OK, or MLA_ERR_DEVICE_TIMEOUT when an in-kernel wait gave up. */
+ * word: MLA_OK, or MLA_ERR_DEVICE_TIMEOUT when an in-kernel wait gave up.  The kernel
+ * that records the first error also writes it to a host-mapped copy, which this call
+ * reads: no device-to-host copy, so it waits for the plan's launches only, not for
+ * copies other streams have queued. */
 mla_status mla_plan_check(mla_plan_t plan);
 
 /* Counts of a plan. */

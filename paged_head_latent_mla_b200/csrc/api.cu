@@ -49,6 +49,7 @@ struct mla_plan_s {
   int64_t uploads = 0;
   size_t blob_cap = 0, ws_cap = 0;  // capacities of the pooled device buffers
   cudaEvent_t ev_last = nullptr;
+  int32_t* h_status = nullptr;  // host-mapped mirror of the status word (see status_slot_take)
   // kernel timing ring (MLA_DEBUG_KERNEL_TIMING): 3 events per run
   static constexpr int kRing = 256;
   cudaEvent_t* ring = nullptr;
@@ -191,6 +192,45 @@ void event_give(int device, cudaEvent_t e) {
   cudaEventDestroy(e);
 }
 
+// Host-visible mirrors of the plans' status words.  The attention kernel that records a
+// plan's first error also stores it here (mapped pinned memory), so mla_plan_check reads
+// it once the launch has finished, with no copy: a synchronous device-to-host copy of the
+// device word would queue behind the device-to-host copies other streams have pending
+// (a serving loop's result downloads) and wait for them.  Slots lie 64 bytes apart in
+// 4 KB slabs that are never freed; the slab's device address must equal its host
+// address (unified addressing).
+std::vector<int32_t*>* g_status_free = new std::vector<int32_t*>();  // never destroyed
+constexpr size_t kStatusSlab = 4096, kStatusStride = 64;
+
+int32_t* status_slot_take() {
+  std::lock_guard<std::mutex> lock(g_pool_mutex);
+  if (g_status_free->empty()) {
+    void* slab = nullptr;
+    void* dev = nullptr;
+    if (cudaHostAlloc(&slab, kStatusSlab, cudaHostAllocPortable | cudaHostAllocMapped) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    if (cudaHostGetDevicePointer(&dev, slab, 0) != cudaSuccess || dev != slab) {
+      cudaGetLastError();
+      cudaFreeHost(slab);
+      return nullptr;
+    }
+    for (size_t off = kStatusSlab; off >= kStatusStride; off -= kStatusStride)
+      g_status_free->push_back(reinterpret_cast<int32_t*>(static_cast<uint8_t*>(slab) + off - kStatusStride));
+  }
+  int32_t* slot = g_status_free->back();
+  g_status_free->pop_back();
+  *reinterpret_cast<volatile int32_t*>(slot) = 0;
+  return slot;
+}
+
+void status_slot_give(int32_t* slot) {
+  if (!slot) return;
+  std::lock_guard<std::mutex> lock(g_pool_mutex);
+  g_status_free->push_back(slot);
+}
+
 // Wait until no launch or upload of the plan can still be reading its buffers.
 void quiesce(mla_plan_s* p) {
   if (p->captured) {
@@ -218,6 +258,7 @@ void free_plan(mla_plan_s* p) {
     pool_give(kPoolDevice, p->device, p->d_blob, p->blob_cap);
     pool_give(kPoolDevice, p->device, p->d_ws, p->ws_cap);
     for (int i = 0; i < 2; ++i) pool_give(kPoolPinned, -1, p->h_staging[i], p->staging_cap[i]);
+    status_slot_give(p->h_status);
   }
   delete p;
 }
@@ -405,6 +446,7 @@ mla_status attention_launch_of(mla_plan_t p, const void* q_nope, const void* q_p
   ap.ws_lse = p->d_ws ? reinterpret_cast<float*>(p->d_ws + static_cast<size_t>(p->sz.cap_ws_rows) * kWsRowOBytes)
                       : nullptr;
   ap.status = p->d_status();
+  ap.status_mirror = p->h_status;
   ap.scale_log2 = p->dims.sm_scale * 1.4426950408889634f;
   ap.num_heads = p->dims.num_heads;
   ap.page_size = p->dims.page_size;
@@ -533,7 +575,7 @@ mla_status mla_plan(const mla_dims* dims, int32_t batch, const int32_t* qo_indpt
     for (int i = 0; i < 3 * mla_plan_s::kRing; ++i)
       if (cudaEventCreate(&p->ring[i]) != cudaSuccess) { cudaGetLastError(); free_plan(p); return MLA_ERR_CUDA; }
   }
-  if (!(p->ev_last = event_take(p->device))) {
+  if (!(p->ev_last = event_take(p->device)) || !(p->h_status = status_slot_take())) {
     free_plan(p);
     return MLA_ERR_CUDA;
   }
@@ -658,13 +700,14 @@ mla_status mla_plan_check(mla_plan_t p) {
   } else if (cudaEventSynchronize(p->ev_last) != cudaSuccess) {
     return MLA_ERR_CUDA;
   }
-  int32_t st = 0;
-  if (cudaMemcpy(&st, p->d_status(), sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return MLA_ERR_CUDA;
+  // the launches have finished: the mirror holds the first error they recorded
+  const int32_t st = *reinterpret_cast<volatile int32_t*>(p->h_status);
   if (st != 0) {
     // The bits above the low byte name the wait that gave up (diagnostics only).
     if (std::getenv("MLA_DEBUG_STATUS")) std::fprintf(stderr, "mla: device status word 0x%x\n", st);
     if (cudaMemset(p->d_status(), 0, sizeof(st)) != cudaSuccess) return MLA_ERR_CUDA;
     if (cudaDeviceSynchronize() != cudaSuccess) return MLA_ERR_CUDA;
+    *reinterpret_cast<volatile int32_t*>(p->h_status) = 0;
     return static_cast<mla_status>(st & 0xff);
   }
   return MLA_OK;

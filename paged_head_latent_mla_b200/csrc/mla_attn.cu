@@ -124,8 +124,15 @@ enum : int32_t {
   kSiteExchange = 11,
 };
 
-__device__ __forceinline__ void record_error(int32_t* status, int32_t site) {
-  atomicCAS(status, 0, MLA_ERR_DEVICE_TIMEOUT | (site << 8));
+// The first error wins the device word; its recorder also copies it to the host-mapped
+// mirror (a plain store: only the winner writes it), which the host reads once the
+// launch has finished without going through a copy engine.
+__device__ __forceinline__ void record_error(int32_t* status, int32_t* mirror, int32_t site) {
+  const int32_t v = MLA_ERR_DEVICE_TIMEOUT | (site << 8);
+  if (atomicCAS(status, 0, v) == 0 && mirror != nullptr) {
+    *reinterpret_cast<volatile int32_t*>(mirror) = v;
+    __threadfence_system();
+  }
 }
 
 }  // namespace attn
@@ -204,7 +211,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     bool good = cluster_scope ? mbar_wait<true>(b, parity, TO, abort_flag) : mbar_wait(b, parity, TO, abort_flag);
     good = __all_sync(0xffffffffu, good);
     if (!good && lane == 0) {
-      record_error(p.status, site);
+      record_error(p.status, p.status_mirror, site);
       *abort_flag = 1;
     }
     return good;
@@ -257,11 +264,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       }
       // Do not leave while our own copies may still be landing.
       if (lane == 0) {
-        if (!mbar_wait(bar(bQFull), 0, TO, abort_flag)) record_error(p.status, kSiteTeardown);
+        if (!mbar_wait(bar(bQFull), 0, TO, abort_flag)) record_error(p.status, p.status_mirror, kSiteTeardown);
         for (int s = 0; s < kStages; ++s)
           if (last_issued[s] >= 0 &&
               !mbar_wait(bar(bKVFull + s), (last_issued[s] / kStages) & 1, TO, abort_flag))
-            record_error(p.status, kSiteTeardown);
+            record_error(p.status, p.status_mirror, kSiteTeardown);
       }
     }
   } else if (warp == kWarpMma) {
@@ -317,7 +324,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       // Every MMA this thread issued must retire before TMEM is released.
       if (lane == 0) {
         mma_commit(bar(bFin));
-        if (!mbar_wait(bar(bFin), 0, TO, abort_flag)) record_error(p.status, kSiteTeardown);
+        if (!mbar_wait(bar(bFin), 0, TO, abort_flag)) record_error(p.status, p.status_mirror, kSiteTeardown);
       }
       __syncwarp();
     }
@@ -342,7 +349,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       }
       if (lane == 0) {
         mma_commit(bar(bFin + 1));
-        if (!mbar_wait(bar(bFin + 1), 0, TO, abort_flag)) record_error(p.status, kSiteTeardown);
+        if (!mbar_wait(bar(bFin + 1), 0, TO, abort_flag)) record_error(p.status, p.status_mirror, kSiteTeardown);
       }
       __syncwarp();
     }

@@ -21,6 +21,7 @@ struct AttnParams {
   void* ws_o;        // bf16 [partials, 128, 512]
   float* ws_lse;     // fp32 [partials, 128]
   int32_t* status;   // device status word
+  int32_t* status_mirror;  // host-mapped pinned copy of the first error recorded, or null
   float scale_log2;  // sm_scale * log2(e)
   float nan_guard;   // always NaN: `x != nan_guard` is true for every x, yet the compiler
                      // cannot fold it, so a vote on it waits for x to be computed

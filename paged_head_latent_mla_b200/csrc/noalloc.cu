@@ -324,6 +324,7 @@ extern "C" mla_status mla_run_noalloc(const mla_dims* dims, int32_t batch, const
   ap.ws_o = partials;
   ap.ws_lse = reinterpret_cast<float*>(partials + size_t(n_ws_rows) * kWsRowOBytes);
   ap.status = reinterpret_cast<int32_t*>(scratch + kOffStatus);
+  ap.status_mirror = nullptr;  // read back by a device-to-device copy below
   ap.scale_log2 = dims->sm_scale * 1.4426950408889634f;
   ap.num_heads = dims->num_heads;
   ap.page_size = dims->page_size;

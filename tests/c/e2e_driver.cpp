@@ -3,8 +3,8 @@
 // from pinned host memory to the device, runs the attention (mla_run), copies the
 // output (and lse) back to pinned host memory, and retires the plan of two steps
 // earlier (mla_plan_check: its device status word; mla_plan_destroy).  Steps are
-// pipelined two deep on three streams (uploads, runs, downloads), each parity with its
-// own device buffers guarded by events, as a serving loop overlaps them.
+// pipelined two deep on three streams (uploads: plan and queries; runs; downloads), each
+// parity with its own device buffers guarded by events, as a serving loop overlaps them.
 //
 //   e2e_driver DIR STEPS WARMUP SM_SCALE
 //
@@ -12,8 +12,8 @@
 // q_nope.bin (bf16 [T][H][512]), q_pe.bin (bf16 [T][H][64]), cache.bin (bf16
 // [num_pages][page_size][576]) and lse (one int32: 1 to download the lse as well).
 // Prints "ms_per_step X", "h2d_bytes_per_step N", "d2h_bytes_per_step N", "status S":
-// the device time from an event before the first timed step's plan to one after its
-// last download, per step.
+// the device time from an event before the first timed step's plan upload to one after
+// its last download, per step.
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -119,7 +119,10 @@ int main(int argc, char** argv) {
   auto one = [&](int i) -> int {
     Buf& b = buf[i & 1];
     mla_plan_t p = nullptr;
-    const mla_status st = mla_plan(&d, batch, qo, kvp, kvi, last, causal, s_run, nullptr, &p);
+    // the plan's upload goes on the upload stream, ahead of the queries: on the compute
+    // stream it would wait for step i-1's run and then queue behind step i+1's query copy
+    // in the copy engine; `uploaded` below orders the run after both
+    const mla_status st = mla_plan(&d, batch, qo, kvp, kvi, last, causal, s_up, nullptr, &p);
     if (st != MLA_OK) return st;
     CK(cudaStreamWaitEvent(s_up, b.computed, 0));  // step i-2 has finished reading these
     CK(cudaMemcpyAsync(b.qn, qn_h, qn_bytes, cudaMemcpyHostToDevice, s_up));
@@ -148,7 +151,7 @@ int main(int argc, char** argv) {
   cudaEvent_t e0, e1;
   CK(cudaEventCreate(&e0));
   CK(cudaEventCreate(&e1));
-  CK(cudaEventRecord(e0, s_run));
+  CK(cudaEventRecord(e0, s_up));
   for (int i = 0; i < steps; ++i)
     if (int r = one(i)) return r;
   for (Buf& b : buf) CK(cudaStreamWaitEvent(s_down, b.downloaded, 0));

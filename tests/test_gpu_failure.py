@@ -3,8 +3,8 @@
 Every wait inside the attention kernel is bounded.  A debug flag makes the kernel skip
 its first key-tile load, so the wait for that tile never completes ("a flag that
 nothing sets"): after the configured timeout the kernel records
-MLA_ERR_DEVICE_TIMEOUT in the plan's status word, every role unwinds, and
-mla_plan_check reports it.  The context stays usable: a normal run afterwards still
+MLA_ERR_DEVICE_TIMEOUT in the plan's status word (and its host-mapped copy), every
+role unwinds, and mla_plan_check reports it.  The context stays usable: a normal run afterwards still
 matches the oracle.
 """
 
@@ -40,6 +40,10 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     M.mla_run(plan, qn, qp, cache, return_lse=True)
     assert M.mla_plan_check(plan) == M.MLA_ERR_DEVICE_TIMEOUT
     assert M.mla_plan_check(plan) == M.MLA_OK  # the status word was cleared
+    # both copies of the word were cleared: the next failing run records and reports again
+    M.mla_run(plan, qn, qp, cache)
+    assert M.mla_plan_check(plan) == M.MLA_ERR_DEVICE_TIMEOUT
+    assert M.mla_plan_check(plan) == M.MLA_OK
     plan.destroy()
     torch.cuda.synchronize(dev)  # no sticky CUDA error
 
