@@ -605,62 +605,77 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
 // M = max_i lse_i, out = sum_i e^{lse_i - M} o_i / sum_i e^{lse_i - M},
 // lse = M + ln sum_i e^{lse_i - M} (FlashInferMLAManager.run: merging key segments).
 // One warp per row; lane l owns columns [16l, 16l + 16), so every load and store of a
-// row is one contiguous 1 KB access; four partials are in flight at a time.
+// row is one contiguous 1 KB access.  Up to eight partials are in flight at a time, and
+// a tile with more than 32 partials is merged 32 at a time against a running maximum.
 __global__ void __launch_bounds__(256) mla_merge_kernel(const MergeParams p) {
-  // Launched as a programmatic dependent of the attention grid: wait until that grid has
-  // finished and its partials are visible.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // The merge list and the reference list are plan data, written before the attention
+  // grid started: read them while that grid drains.
   const MergeItem m = p.merge[blockIdx.x >> 4];  // 16 blocks per split query tile
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = ((blockIdx.x & 15) << 3) + warp;  // 8 rows (one per warp) per block
   if (r >= m.n_rows) return;
-  const float neg_inf = -__int_as_float(0x7f800000);
   const int n = m.n_refs;
   const int32_t* refs = p.refs + m.first_ref;  // workspace row of each partial's row 0
-  float M = neg_inf;
-  for (int i = lane; i < n; i += 32) M = fmaxf(M, p.ws_lse[static_cast<size_t>(refs[i]) + r]);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  int ref_l = lane < n ? refs[lane] : 0;       // lane u holds partial u's reference (u < 32)
+  // Launched as a programmatic dependent of the attention grid: wait until that grid has
+  // finished and its partials are visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const float neg_inf = -__int_as_float(0x7f800000);
   float acc[16];
 #pragma unroll
   for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-  float z = 0.f;
-  if (M != neg_inf) {
-    for (int i0 = 0; i0 < n; i0 += 32) {
-      const int cnt = min(32, n - i0);
-      // lane u holds the weight of partial i0 + u
-      const int ref_l = lane < cnt ? refs[i0 + lane] : 0;
-      const float wl = lane < cnt ? __expf(p.ws_lse[static_cast<size_t>(ref_l) + r] - M) : 0.f;
-      z += wl;
-      for (int k = 0; k < cnt; k += 4) {
-        uint4 v[4][2];
-        float wk[4];
+  float M = neg_inf, z = 0.f;
+  for (int i0 = 0; i0 < n; i0 += 32) {
+    const int cnt = min(32, n - i0);
+    if (i0 > 0) ref_l = lane < cnt ? refs[i0 + lane] : 0;
+    const float l_l = lane < cnt ? p.ws_lse[static_cast<size_t>(ref_l) + r] : neg_inf;
+    // every partial of this group in flight before any is used (8 at a time)
+    for (int k = 0; k < cnt; k += 8) {
+      uint4 v[8][2];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          wk[u] = __shfl_sync(0xffffffffu, wl, k + u);  // k + u <= 31
-          const int ref_u = __shfl_sync(0xffffffffu, ref_l, k + u);
-          if (k + u < cnt) {
-            const uint4* src = reinterpret_cast<const uint4*>(
-                static_cast<const uint8_t*>(p.ws_o) + ((static_cast<size_t>(ref_u) + r) * kCkv + 16 * lane) * 2);
-            v[u][0] = src[0];
-            v[u][1] = src[1];
-          } else {
-            v[u][0] = v[u][1] = make_uint4(0u, 0u, 0u, 0u);
-          }
+      for (int u = 0; u < 8; ++u) {
+        const int ref_u = __shfl_sync(0xffffffffu, ref_l, (k + u) & 31);
+        if (k + u < cnt) {
+          const uint4* src = reinterpret_cast<const uint4*>(
+              static_cast<const uint8_t*>(p.ws_o) + ((static_cast<size_t>(ref_u) + r) * kCkv + 16 * lane) * 2);
+          v[u][0] = src[0];
+          v[u][1] = src[1];
+        } else {
+          v[u][0] = v[u][1] = make_uint4(0u, 0u, 0u, 0u);
         }
+      }
+      if (k == 0) {
+        // the group's running max; earlier groups' sums are rescaled to it
+        float Mg = l_l;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint32_t* wv = reinterpret_cast<const uint32_t*>(v[u]);
+        for (int off = 16; off > 0; off >>= 1) Mg = fmaxf(Mg, __shfl_xor_sync(0xffffffffu, Mg, off));
+        const float Mn = fmaxf(M, Mg);
+        if (Mn != neg_inf && M != neg_inf && Mn != M) {
+          const float s = __expf(M - Mn);
+          z *= s;
 #pragma unroll
-          for (int k2 = 0; k2 < 8; ++k2) {
-            acc[2 * k2] += wk[u] * __uint_as_float(wv[k2] << 16);
-            acc[2 * k2 + 1] += wk[u] * __uint_as_float(wv[k2] & 0xffff0000u);
-          }
+          for (int q = 0; q < 16; ++q) acc[q] *= s;
+        }
+        M = Mn;
+      }
+      const float wl = (lane < cnt && M != neg_inf) ? __expf(l_l - M) : 0.f;
+      if (k == 0) {
+        float zg = wl;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) zg += __shfl_xor_sync(0xffffffffu, zg, off);
+        z += zg;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float wk = __shfl_sync(0xffffffffu, wl, (k + u) & 31);
+        const uint32_t* wv = reinterpret_cast<const uint32_t*>(v[u]);
+#pragma unroll
+        for (int k2 = 0; k2 < 8; ++k2) {
+          acc[2 * k2] += wk * __uint_as_float(wv[k2] << 16);
+          acc[2 * k2 + 1] += wk * __uint_as_float(wv[k2] & 0xffff0000u);
         }
       }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
   }
   const float inv = z > 0.f ? 1.f / z : 0.f;
   uint4 o[2];

@@ -337,3 +337,13 @@ def test_opposite_half_partials():
     d.cache, d.q_nope, d.q_pe = c.to(torch.bfloat16), qn.to(torch.bfloat16), qp.to(torch.bfloat16)
     out, lse, _, _ = gpu_run(d)
     compare(d, out, lse)
+
+
+@pytest.mark.parametrize("kv", [[2100, 300], [4500, 64]])
+def test_merge_of_many_partials(kv):
+    """Split tiles with more than 32 partials (33 and 71 chunks of 64 keys): the merge
+    takes them 32 at a time against a running maximum of their log-sum-exps."""
+    d = make_custom([2, 1], kv, 64, 64, seed=13)
+    out, lse, info, _ = gpu_run(d, split_keys=64)
+    assert info["num_merge_refs"] > 32
+    compare(d, out, lse)
