@@ -71,3 +71,23 @@ def test_launch_errors_are_status_codes_not_exceptions():
     assert lib.mla_run(plan.handle, None, qp.data_ptr(), cache.data_ptr(), out.data_ptr(), None, None) == \
         M.MLA_ERR_INVALID_ARGUMENT
     plan.destroy()
+
+
+def test_status_slots_are_per_plan():
+    """Each plan's host-mapped status copy is its own: with 150 plans alive (more than
+    one 64-slot slab), a timeout in one is reported by that plan only, and every other
+    plan reports OK; slots of destroyed plans are reused clean."""
+    dev = torch.device("cuda:0")
+    d = make_custom([1], [200], 16, 16, seed=53)
+    qn, qp, cache = d.q_nope.to(dev), d.q_pe.to(dev), d.cache.to(dev)
+    for _round in range(2):
+        plans = [_plan(d) for _ in range(150)]
+        bad = _plan(d, debug_flags=M.MLA_DEBUG_DROP_FIRST_KV_LOAD, wait_timeout_ns=50_000_000)
+        plans.insert(75, bad)
+        for p in plans:
+            M.mla_run(p, qn, qp, cache)
+        for p in plans:
+            assert M.mla_plan_check(p) == (M.MLA_ERR_DEVICE_TIMEOUT if p is bad else M.MLA_OK)
+        for p in plans:
+            p.destroy()
+    torch.cuda.synchronize(dev)
