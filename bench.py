@@ -472,7 +472,7 @@ def time_e2e(d, device, steps, warmup):
     return ms, h2d[0], d2h
 
 
-def time_e2e_cpp(d, steps, warmup):
+def time_e2e_cpp(d, steps, warmup, device_index=0):
     """The same end-to-end loop as time_e2e, written as a C++ client of the C ABI
     (tests/c/e2e_driver.cpp): per step mla_plan from host tables, H2D of the queries from
     pinned memory, mla_run, D2H of the result to pinned memory, pipelined two deep on
@@ -507,8 +507,8 @@ def time_e2e_cpp(d, steps, warmup):
                 f.write(t.contiguous().view(torch.int16).numpy().tobytes())
         with open(os.path.join(tmp, "lse"), "wb") as f:
             f.write(np.array([1 if d.return_lse else 0], np.int32).tobytes())
-        r = subprocess.run([exe, tmp, str(steps), str(warmup), repr(float(d.sm_scale))], capture_output=True,
-                           text=True, timeout=300)
+        r = subprocess.run([exe, tmp, str(steps), str(warmup), repr(float(d.sm_scale)), str(device_index)],
+                           capture_output=True, text=True, timeout=300)
         if r.returncode != 0:
             return {"error": f"rc {r.returncode}: {r.stderr[-300:]}"}
         out = dict(line.split() for line in r.stdout.strip().splitlines())
@@ -852,7 +852,7 @@ def run_native(args):
         e2e_python = {"value": job_throughput(w["kv_bytes"], world, py_ms), "unit": "GB/s",
                       "h2d_bytes_per_step": int(py_h2d), "d2h_bytes_per_step": int(py_d2h), "ms_per_step": py_ms,
                       "client": "Python binding (paged_head_latent_mla_b200)"}
-        cpp = time_e2e_cpp(d, e2e_steps, 3)
+        cpp = time_e2e_cpp(d, e2e_steps, 3, device_index=device.index)
         # every rank takes the same collective steps: a failed C++ run reports inf
         cpp_ms = reduce_max_over_ranks(cpp[0] if isinstance(cpp, tuple) else float("inf"), dist, device)
         if isinstance(cpp, tuple) and cpp_ms != float("inf"):

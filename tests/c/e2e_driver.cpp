@@ -6,7 +6,7 @@
 // pipelined two deep on three streams (uploads: plan and queries; runs; downloads), each
 // parity with its own device buffers guarded by events, as a serving loop overlaps them.
 //
-//   e2e_driver DIR STEPS WARMUP SM_SCALE
+//   e2e_driver DIR STEPS WARMUP SM_SCALE [DEVICE]
 //
 // DIR holds: tables (one step's tables in the int32 layout of plan_timer.cpp),
 // q_nope.bin (bf16 [T][H][512]), q_pe.bin (bf16 [T][H][64]), cache.bin (bf16
@@ -58,7 +58,9 @@ int main(int argc, char** argv) {
   const std::string dir = argv[1];
   const int steps = std::atoi(argv[2]), warmup = std::atoi(argv[3]);
   const float sm_scale = static_cast<float>(std::atof(argv[4]));
+  const int device = argc > 5 ? std::atoi(argv[5]) : 0;
   if (steps < 1 || warmup < 0) return 2;
+  CK(cudaSetDevice(device));
   std::vector<unsigned char> tab, qn_f, qp_f, cache_f, lse_f;
   if (!read_file(dir + "/tables", &tab) || !read_file(dir + "/q_nope.bin", &qn_f) ||
       !read_file(dir + "/q_pe.bin", &qp_f) || !read_file(dir + "/cache.bin", &cache_f) ||
