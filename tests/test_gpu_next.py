@@ -523,3 +523,44 @@ def test_random_steps_match_oracle(c):
                                    d.last_page_len, c["P"], d.sm_scale, causal=c["causal"],
                                    context_only=c["context_only"])
     _check(out, lse, ref_o, ref_l)
+
+
+def test_cpp_end_to_end_client(tmp_path):
+    """The C++ serving loop the benchmark times (tests/c/e2e_driver.cpp) runs on the GPU
+    through the C ABI: every step plans from host tables, uploads its queries from pinned
+    memory, runs, downloads the result and lse, and retires the plan of two steps earlier
+    through mla_plan_check; it ends with status 0 and reports the bytes it moved."""
+    import os
+    import shutil
+    import subprocess
+
+    cxx = shutil.which("g++") or shutil.which("c++")
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    if cxx is None or not os.path.exists(os.path.join(cuda, "include", "cuda_runtime.h")):
+        pytest.skip("no C++ compiler or CUDA headers")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    lib_dir = os.path.dirname(M.LIB_PATH)
+    exe = str(tmp_path / "e2e_driver")
+    r = subprocess.run([cxx, "-O2", "-std=c++17", "-I", os.path.join(root, "include"), "-I",
+                        os.path.join(cuda, "include"), os.path.join(root, "tests", "c", "e2e_driver.cpp"), "-L",
+                        lib_dir, "-l:libmla_b200.so", "-L", os.path.join(cuda, "lib64"), "-lcudart",
+                        "-Wl,-rpath," + lib_dir + ":" + os.path.join(cuda, "lib64"), "-o", exe],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    d = make_custom([1, 3, 2], [700, 90, 1500], 64, 32, seed=71)
+    hdr = np.array([d.num_heads, d.page_size, d.num_pages, d.batch, 1], np.int32)
+    with open(tmp_path / "tables", "wb") as f:
+        for a in (hdr, d.qo_indptr.numpy(), d.kv_indptr.numpy(), d.kv_indices.numpy(), d.last_page_len.numpy()):
+            f.write(np.ascontiguousarray(a, dtype=np.int32).tobytes())
+    for name, t in (("q_nope.bin", d.q_nope), ("q_pe.bin", d.q_pe), ("cache.bin", d.cache)):
+        (tmp_path / name).write_bytes(t.contiguous().view(torch.int16).numpy().tobytes())
+    (tmp_path / "lse").write_bytes(np.array([1], np.int32).tobytes())
+    r = subprocess.run([exe, str(tmp_path), "6", "2", repr(float(d.sm_scale)), "0"], capture_output=True, text=True,
+                       timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    got = dict(line.split() for line in r.stdout.strip().splitlines())
+    T, H = d.total_tokens, d.num_heads
+    assert int(got["status"]) == 0
+    assert float(got["ms_per_step"]) > 0
+    assert int(got["d2h_bytes_per_step"]) == T * H * 512 * 2 + T * H * 4
+    assert int(got["h2d_bytes_per_step"]) > T * H * 576 * 2  # the queries and the plan's upload
