@@ -66,13 +66,22 @@ int main(int argc, char** argv) {
       !read_file(dir + "/q_pe.bin", &qp_f) || !read_file(dir + "/cache.bin", &cache_f) ||
       !read_file(dir + "/lse", &lse_f))
     return 2;
+  // every size is checked against the tables' header before anything is read
+  const size_t n32 = tab.size() / 4;
+  if (n32 < 5) return 2;
   const int32_t* t32 = reinterpret_cast<const int32_t*>(tab.data());
   const int32_t H = t32[0], P = t32[1], pages = t32[2], batch = t32[3], causal = t32[4];
+  if (H <= 0 || P <= 0 || pages <= 0 || batch < 0 || n32 < 5 + 2 * (static_cast<size_t>(batch) + 1)) return 2;
   const int32_t* qo = t32 + 5;
   const int32_t* kvp = qo + batch + 1;
+  if (kvp[batch] < 0 || n32 != 5 + 2 * (static_cast<size_t>(batch) + 1) + static_cast<size_t>(kvp[batch]) + batch)
+    return 2;
   const int32_t* kvi = kvp + batch + 1;
   const int32_t* last = kvi + kvp[batch];
   const int32_t T = qo[batch];
+  if (T < 0 || qn_f.size() != static_cast<size_t>(T) * H * 512 * 2 || qp_f.size() != static_cast<size_t>(T) * H * 64 * 2 ||
+      cache_f.size() != static_cast<size_t>(pages) * P * 576 * 2)
+    return 2;
   const bool want_lse = lse_f.size() >= 4 && *reinterpret_cast<const int32_t*>(lse_f.data()) != 0;
   const size_t qn_bytes = qn_f.size(), qp_bytes = qp_f.size();
   const size_t out_bytes = static_cast<size_t>(T) * H * 512 * 2, lse_bytes = static_cast<size_t>(T) * H * 4;
