@@ -347,3 +347,14 @@ def test_merge_of_many_partials(kv):
     out, lse, info, _ = gpu_run(d, split_keys=64)
     assert info["num_merge_refs"] > 32
     compare(d, out, lse)
+
+
+def test_very_long_row():
+    """One decode token over 262,144 keys (4096 pages, 302 MB of cache) next to a short
+    row: the planner spreads the long row over many work items, so its query tile is
+    merged from more than 32 partials (the merge's running-maximum path at scale), and
+    page and key indices reach their largest values in the suite.  Compared in full."""
+    d = make_custom([1, 1], [262_144, 300], 128, 64, seed=31)
+    out, lse, info, _ = gpu_run(d)
+    assert info["num_merge"] >= 1 and info["num_merge_refs"] > 32
+    compare(d, out, lse)
