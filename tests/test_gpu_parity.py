@@ -371,3 +371,14 @@ def test_large_batch_of_short_rows():
     out, lse, info, _ = gpu_run(d)
     assert info["num_work"] >= 2048
     compare(d, out, lse, tokens=list(range(0, 2048, 8)) + [2047])
+
+
+def test_long_causal_prefill_small_heads():
+    """A 1000-token causal prefill over 3000 keys at 16 heads (8 tokens per query tile, so
+    the causal edge runs through every tile) in 128-key pages, beside a decode row:
+    every 7th token, the first and last of the row, and the tokens around tile edges are
+    compared with the oracle."""
+    d = make_custom([1000, 1], [3000, 2222], 16, 128, seed=41)
+    out, lse, _, _ = gpu_run(d)
+    toks = set(range(0, 1000, 7)) | {0, 999, 1000} | {t for b in range(8, 1000, 128) for t in (b - 1, b)}
+    compare(d, out, lse, tokens=sorted(toks))
